@@ -1,0 +1,122 @@
+"""fp64 CPU oracle for the KDA gated delta-rule recurrence.
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, by ``__graft_entry__.smoke()``
+and by the CPU-baseline leg of ``bench.py``. The CUDA library never imports,
+links or calls anything here, and nothing here imports the CUDA library.
+
+The C source (``kda_oracle.c``) runs the recurrence one token at a time in
+fp64 (pages: "22580: from GPT-2 to Kimi K3, explained", sections "DeltaNet,
+or Fast Weight Programmers" (cached forward), "Gated Delta Net" (the decay
+alpha) and "KDA / Kimi Linear" (one decay per key channel)):
+
+    S' = Diag(exp(log_alpha_t)) S;  r = S'^T k_t;  d = beta_t (v_t - r)
+    S  = S' + k_t d^T;              o_t = S^T q_t
+
+Inputs of any float dtype (bf16, fp32, fp64) are widened exactly to fp64
+before the call, so the oracle sees precisely the values the GPU sees.
+
+Pins (tests/test_oracle_pins.py) tie it to what the pages and mathematics
+fix: the no-change, overwrite/retrieval, clear and no-update invariants, the
+unrolled Householder product form, the ungated and gated chunk algebra, and
+split/resume equivalence.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from .build import build as _build
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build()
+        lib = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        lib.oracle_kda_forward.argtypes = [
+            dp, dp, dp, dp, dp, dp, ctypes.POINTER(ctypes.c_int64),
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            dp, dp, ctypes.c_int]
+        lib.oracle_kda_forward.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(x):
+    """Exact widening to a contiguous fp64 numpy array (torch or numpy in)."""
+    if x is None:
+        return None
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().to("cpu", torch.float64).contiguous().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def default_threads() -> int:
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+def kda_forward(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None,
+                n_threads=None):
+    """Run the recurrence over packed sequences.
+
+    q, k, log_alpha: [T_total, H, dk]; v: [T_total, H, dv]; beta: [T_total, H];
+    init_state: [N, H, dk, dv] or None (zeros); cu_seqlens: [N+1] or None
+    (one sequence of T_total tokens). Batched inputs [B, T, H, d] are accepted
+    and treated as B sequences of T tokens. Returns (o, final_state) in fp64,
+    o shaped like v.
+    """
+    q, k, v, la, b = map(_f64, (q, k, v, log_alpha, beta))
+    s0 = _f64(init_state)
+    out_shape = v.shape
+    if q.ndim == 4:  # [B, T, H, d] -> packed
+        B, T = q.shape[:2]
+        if cu_seqlens is None:
+            cu_seqlens = np.arange(B + 1, dtype=np.int64) * T
+        q, k, v, la = (x.reshape(B * T, *x.shape[2:]) for x in (q, k, v, la))
+        b = b.reshape(B * T, -1)
+    T_total, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens is None:
+        cu_seqlens = np.array([0, T_total], dtype=np.int64)
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    n_seq = cu.shape[0] - 1
+    if cu[-1] != T_total:
+        raise ValueError("cu_seqlens[-1] must equal the number of tokens")
+    for x, shp in ((k, (T_total, H, dk)), (la, (T_total, H, dk)),
+                   (v, (T_total, H, dv)), (b, (T_total, H))):
+        if x.shape != shp:
+            raise ValueError("shape mismatch: %s vs %s" % (x.shape, shp))
+    if s0 is not None and s0.shape != (n_seq, H, dk, dv):
+        raise ValueError("init_state must be [N, H, dk, dv]")
+    o = np.zeros((T_total, H, dv), dtype=np.float64)
+    fin = np.zeros((n_seq, H, dk, dv), dtype=np.float64)
+    nt = default_threads() if n_threads is None else int(n_threads)
+    rc = _load().oracle_kda_forward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(s0),
+        cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+        n_seq, H, dk, dv, _ptr(o), _ptr(fin), nt)
+    if rc != 0:
+        raise RuntimeError("oracle_kda_forward failed with code %d" % rc)
+    return o.reshape(out_shape), fin
+
+
+def kda_decode_step(q, k, v, log_alpha, beta, state):
+    """One decode step for B sequences: q, k, log_alpha [B, H, dk]; v [B, H, dv];
+    beta [B, H]; state [B, H, dk, dv]. Returns (o [B, H, dv], new state)."""
+    q, k, v, la, b = map(_f64, (q, k, v, log_alpha, beta))
+    B = q.shape[0]
+    cu = np.arange(B + 1, dtype=np.int64)
+    return kda_forward(q, k, v, la, b, init_state=state, cu_seqlens=cu)
