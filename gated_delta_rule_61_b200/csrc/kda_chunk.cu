@@ -1,0 +1,601 @@
+// kda_chunk.cu -- chunked KDA prefill on sm_100a tensor cores (tcgen05 MMAs,
+// tensor-memory accumulators), chunk C = 64, dk = dv = 128, bf16 inputs.
+//
+// Method. Pages: "22580: from GPT-2 to Kimi K3, explained", section "DeltaNet,
+// or Parallelizing Linear Transformers with Delta Rule" (cut the sequence into
+// chunks of C tokens; inside a chunk the deltas come from a unit lower-
+// triangular system built from the keys (the UT/WY form of the Householder
+// products), across chunks the state carries everything: "C = 64 or 128 ...
+// tensor-core instructions such as UMMA"), with the per-channel decay of
+// "Gated Delta Net" (cumulative decay is a multiplicative prefix sum) and
+// "KDA / Kimi Linear"; the ai-flip.ru KDA explainer (channel-wise diagonal
+// gate; chunked computation on tensor cores). Derived for the KDA step
+// S_t = (I - b k k^T) Diag(a_t) S_{t-1} + b k v^T, with g the within-chunk
+// cumulative sum of log_alpha per key channel and S0 the state entering the
+// chunk:
+//   M_kk[r,j] = sum_c k_rc k_jc e^{g_rc - g_jc} (j < r)
+//   M_qk[r,j] = sum_c q_rc k_jc e^{g_rc - g_jc} (j <= r)
+//   X = (I + diag(beta) M_kk)^-1,  T = X diag(beta)
+//   W = T (K * e^g),  U = T V,  D = U - W S0
+//   O = (Q * e^g) S0 + M_qk D
+//   S1 = Diag(e^{g_last}) S0 + (K * e^{g_last - g})^T D
+//
+// Gram products. e^{g_r - g_j} is split as (x_r e^{g_r - m_a})(k_j e^{m_a - g_j})
+// with m_a the midpoint of the cumulative gate over the row's 16-token
+// sub-chunk a: for j in the same sub-chunk both factors are at most
+// e^{(15/2) * 10} (log_alpha is clamped to >= -10 here), and for j in an
+// earlier sub-chunk the right factor is at most 1. One 128 x 160 x 128 bf16
+// MMA computes all of it: A = [k rows; q rows] scaled by e^{g - m_a}, B = [E;
+// R1; R2; R3] with E_j = k_j e^{m_(sub(j)) - g_j} (diagonal blocks) and
+// R_a rows = k_j e^{m_a - g_j} for j < 16 a (off-diagonal blocks of rows in
+// sub-chunk a). Entries outside the blocks each row needs are ignored.
+//
+// Precision. Gram, T, W, U and the products with the state S0 use bf16
+// operands with fp32 accumulation; the state update (K^T D) and the
+// output's correction (M_qk D) read D straight from tensor memory as tf32,
+// and the state itself stays fp32 in tensor memory for the whole sequence.
+//
+// Layout. One CTA (256 threads) per (sequence, head) chain, walking its
+// chunks in order. Tensor memory (512 columns, lanes = dv index m for the
+// state-sized accumulators):
+//   [0,128)   S^T (fp32 state, lane m, column c)
+//   [128,192) U^T, then D^T = U^T - (W S0)^T   (lane m, column = position)
+//   [192,256) O^T                              (lane m, column = position)
+//   [256,416) Gram result (lanes 0..63 k rows, 64..127 q rows); later W^T
+// Per chunk: (P1) gates and operand tiles from global memory; (P2) Gram MMA;
+// (P3) rows of M_kk and M_qk out of tensor memory; (P4) block forward
+// substitution for X on CUDA cores; (P5) W^T and U^T MMAs; (P6) -W to shared
+// memory, S0 to bf16 and the decay of the fp32 state; (P7) D and the first
+// part of O; (P8) tf32 state update and output correction; (P9) O to HBM.
+#include "kda_common.cuh"
+#include "kda_tc.cuh"
+
+namespace kda {
+namespace chunk64 {
+
+constexpr int C = 64, DK = 128, DV = 128;
+constexpr int kThreads = 256;
+constexpr float kLogAlphaMin = -10.0f;
+constexpr uint64_t kMaxWaitNs = 1000000000ull;  // 1 s per bounded wait
+
+// Shared memory (byte offsets from a 1024-aligned base).
+constexpr uint32_t OFF_SB = 0;         // S0 bf16, K-major [m][c]            32768
+constexpr uint32_t OFF_QT = 32768;     // Q*e^g bf16, K-major [r][c]          16384
+constexpr uint32_t OFF_KT = 49152;     // K*e^(glast-g) fp32, K-major [c][j]  32768
+constexpr uint32_t OFF_BK = 81920;     // K*e^g bf16, MN-major [j][c]         16384
+constexpr uint32_t OFF_VV = 98304;     // V bf16, MN-major [j][m]             16384
+constexpr uint32_t OFF_AG = 114688;    // Gram A bf16 K-major [128][c]        32768
+constexpr uint32_t OFF_MQK = OFF_AG;           // after the Gram MMA: M_qk fp32 K-major [r][j]
+constexpr uint32_t OFF_TM = OFF_AG + 16384;    // T bf16 K-major [r][j]
+constexpr uint32_t OFF_BG = 147456;    // Gram B bf16 K-major [160][c]        40960
+constexpr uint32_t OFF_NMAT = OFF_BG;          // after the Gram MMA: diag(beta) M_kk, fp32 [64][65]
+constexpr uint32_t OFF_XMAT = OFF_BG + 16640;  // X, fp32 [64][65]
+constexpr uint32_t OFF_YBUF = OFF_BG + 33280;  // block products, fp32 [3][16][17]
+constexpr uint32_t OFF_NW = OFF_BG;            // after the solve: -W^T bf16 MN-major [c][r]
+constexpr uint32_t OFF_MISC = 188416;
+constexpr uint32_t MISC_GAMMA = 0, MISC_BETA = 512, MISC_TOT = 768, MISC_MID = 2816,
+                   MISC_GLAST = 4864, MISC_MBAR = 5376, MISC_TMEM = 5384;
+constexpr uint32_t kSmemBytes = OFF_MISC + 5392 + 1024;
+
+// Tensor-memory columns.
+constexpr uint32_t TM_S = 0, TM_D = 128, TM_O = 192, TM_G = 256, TM_W = 256;
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&p);
+}
+
+// All threads wait for the MMA barrier phase; thread 0 spins (bounded) and
+// the result is shared through the CTA barrier.
+__device__ __forceinline__ bool cta_wait(uint32_t mbar, uint32_t parity, int code) {
+  int fail = 0;
+  if (threadIdx.x == 0) fail = !tc::mbar_wait_bounded(mbar, parity, kMaxWaitNs) ? 1 : 0;
+  fail = __syncthreads_or(fail);
+  tc::fence_after_sync();
+  if (fail && threadIdx.x == 0) report_timeout(code);
+  return fail == 0;
+}
+
+__device__ __forceinline__ void cta_sync_tc() {
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+               const __nv_bfloat16* __restrict__ v, const float* __restrict__ log_alpha,
+               const float* __restrict__ beta, const float* __restrict__ init_state,
+               const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ order,
+               int T, int H, __nv_bfloat16* __restrict__ o, float* __restrict__ final_state) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = tc::smem_u32(smem);
+  float* s_gamma = reinterpret_cast<float*>(smem + OFF_MISC + MISC_GAMMA);
+  float* s_beta = reinterpret_cast<float*>(smem + OFF_MISC + MISC_BETA);
+  float* s_tot = reinterpret_cast<float*>(smem + OFF_MISC + MISC_TOT);
+  float* s_mid = reinterpret_cast<float*>(smem + OFF_MISC + MISC_MID);
+  float* s_glast = reinterpret_cast<float*>(smem + OFF_MISC + MISC_GLAST);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC + MISC_TMEM);
+  const uint32_t mbar = sbase + OFF_MISC + MISC_MBAR;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int chain = blockIdx.x;
+  const int seq = order ? order[chain / H] : chain / H;
+  const int head = chain % H;
+  long long t_begin, t_end;
+  seq_bounds(cu_seqlens, seq, T, &t_begin, &t_end);
+
+  if (warp == 0) {
+    tc::tmem_alloc(tc::smem_u32(tmem_slot), 512);
+    tc::tmem_relinquish();
+  }
+  if (tid == 0) {
+    tc::mbar_init(mbar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  cta_sync_tc();
+  const uint32_t tmem = *tmem_slot;
+  uint32_t phase = 0;
+  bool ok = true;
+
+  // TMEM access: warp w reaches lanes [32 (w % 4), +32); the two warps that
+  // share a lane quadrant split the columns of 128-column passes.
+  const int quad = warp & 3, half = warp >> 2;
+  const int m = quad * 32 + lane;
+  const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+  const size_t state_off = ((size_t)seq * H + head) * DK * DV;
+
+  // Initial state: S^T[m][c] = S0[c][m].
+  {
+    const uint32_t tb = tmem + lane_off + TM_S + half * 64;
+#pragma unroll
+    for (int cg = 0; cg < 4; ++cg) {
+      float vals[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int c = half * 64 + cg * 16 + i;
+        vals[i] = init_state ? init_state[state_off + (size_t)c * DV + m] : 0.f;
+      }
+      tc::tmem_st16(tb + cg * 16, vals);
+    }
+    tc::tmem_wait_st();
+  }
+  cta_sync_tc();
+
+  const long long len = t_end - t_begin;
+  const int n_chunks = (int)((len + C - 1) / C);
+  const int pr = tid & 63, sub = tid >> 6, c0 = 2 * pr;  // P1 mapping
+
+  for (int n = 0; n < n_chunks; ++n) {
+    const long long t0 = t_begin + (long long)n * C;
+    const int L = (int)((t_end - t0) < C ? (t_end - t0) : C);
+
+    // ---- P1: cumulative gates and operand tiles --------------------------
+    float g0[16], g1[16];
+    {
+      float run0 = 0.f, run1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int r = sub * 16 + i;
+        float2 l = make_float2(0.f, 0.f);
+        if (r < L)
+          l = __ldg(reinterpret_cast<const float2*>(
+              log_alpha + ((size_t)(t0 + r) * H + head) * DK + c0));
+        run0 += fmaxf(l.x, kLogAlphaMin);
+        run1 += fmaxf(l.y, kLogAlphaMin);
+        g0[i] = run0;
+        g1[i] = run1;
+      }
+      s_tot[sub * 128 + c0] = run0;
+      s_tot[sub * 128 + c0 + 1] = run1;
+    }
+    __syncthreads();
+    float m0, m1;
+    {
+      float off0 = 0.f, off1 = 0.f;
+      for (int b = 0; b < sub; ++b) {
+        off0 += s_tot[b * 128 + c0];
+        off1 += s_tot[b * 128 + c0 + 1];
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        g0[i] += off0;
+        g1[i] += off1;
+      }
+      m0 = 0.5f * (g0[0] + g0[15]);
+      m1 = 0.5f * (g1[0] + g1[15]);
+      s_mid[sub * 128 + c0] = m0;
+      s_mid[sub * 128 + c0 + 1] = m1;
+      if (sub == 3) {
+        s_glast[c0] = g0[15];
+        s_glast[c0 + 1] = g1[15];
+        s_gamma[c0] = expf(g0[15]);
+        s_gamma[c0 + 1] = expf(g1[15]);
+      }
+    }
+    __syncthreads();
+    {
+      const float em0 = expf(m0), em1 = expf(m1);
+      const float kt0 = expf(s_glast[c0] - m0), kt1 = expf(s_glast[c0 + 1] - m1);
+      float rho0[4], rho1[4];
+#pragma unroll
+      for (int ap = 0; ap < 4; ++ap) {
+        rho0[ap] = ap > sub ? expf(s_mid[ap * 128 + c0] - m0) : 0.f;
+        rho1[ap] = ap > sub ? expf(s_mid[ap * 128 + c0 + 1] - m1) : 0.f;
+      }
+      float kt_c0[16], kt_c1[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int r = sub * 16 + i;
+        float k0 = 0.f, k1 = 0.f, q0 = 0.f, q1 = 0.f, v0 = 0.f, v1 = 0.f, bt = 0.f;
+        if (r < L) {
+          const size_t tok = (size_t)(t0 + r) * H + head;
+          const float2 kk = __bfloat1622float2(
+              *reinterpret_cast<const __nv_bfloat162*>(k + tok * DK + c0));
+          const float2 qq = __bfloat1622float2(
+              *reinterpret_cast<const __nv_bfloat162*>(q + tok * DK + c0));
+          const float2 vv = __bfloat1622float2(
+              *reinterpret_cast<const __nv_bfloat162*>(v + tok * DV + c0));
+          k0 = kk.x; k1 = kk.y; q0 = qq.x; q1 = qq.y; v0 = vv.x; v1 = vv.y;
+          bt = __ldg(beta + tok);
+        }
+        if (pr == 0) s_beta[r] = bt;
+        const float f0 = __expf(g0[i] - m0), f1 = __expf(g1[i] - m1);
+        const float fi0 = __expf(m0 - g0[i]), fi1 = __expf(m1 - g1[i]);
+        *reinterpret_cast<uint32_t*>(smem + OFF_AG + tc::sw128<2>(r, c0, 128)) =
+            pack_bf16x2(k0 * f0, k1 * f1);
+        *reinterpret_cast<uint32_t*>(smem + OFF_AG + tc::sw128<2>(64 + r, c0, 128)) =
+            pack_bf16x2(q0 * f0, q1 * f1);
+        const float e0 = k0 * fi0, e1 = k1 * fi1;
+        *reinterpret_cast<uint32_t*>(smem + OFF_BG + tc::sw128<2>(r, c0, 160)) =
+            pack_bf16x2(e0, e1);
+        if (sub < 1)
+          *reinterpret_cast<uint32_t*>(smem + OFF_BG + tc::sw128<2>(64 + r, c0, 160)) =
+              pack_bf16x2(e0 * rho0[1], e1 * rho1[1]);
+        if (sub < 2)
+          *reinterpret_cast<uint32_t*>(smem + OFF_BG + tc::sw128<2>(80 + r, c0, 160)) =
+              pack_bf16x2(e0 * rho0[2], e1 * rho1[2]);
+        if (sub < 3)
+          *reinterpret_cast<uint32_t*>(smem + OFF_BG + tc::sw128<2>(112 + r, c0, 160)) =
+              pack_bf16x2(e0 * rho0[3], e1 * rho1[3]);
+        const float eg0 = f0 * em0, eg1 = f1 * em1;
+        *reinterpret_cast<uint32_t*>(smem + OFF_QT + tc::sw128<2>(r, c0, 64)) =
+            pack_bf16x2(q0 * eg0, q1 * eg1);
+        *reinterpret_cast<uint32_t*>(smem + OFF_BK + tc::sw128<2>(r, c0, 64)) =
+            pack_bf16x2(k0 * eg0, k1 * eg1);
+        *reinterpret_cast<uint32_t*>(smem + OFF_VV + tc::sw128<2>(r, c0, 64)) =
+            pack_bf16x2(v0, v1);
+        kt_c0[i] = e0 * kt0;
+        kt_c1[i] = e1 * kt1;
+      }
+      // K~ as a K-major tf32 operand [c][j]: 16 consecutive positions per channel.
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const int j = sub * 16 + q4 * 4;
+        *reinterpret_cast<float4*>(smem + OFF_KT + tc::sw128<4>(c0, j, 128)) =
+            make_float4(kt_c0[q4 * 4], kt_c0[q4 * 4 + 1], kt_c0[q4 * 4 + 2], kt_c0[q4 * 4 + 3]);
+        *reinterpret_cast<float4*>(smem + OFF_KT + tc::sw128<4>(c0 + 1, j, 128)) =
+            make_float4(kt_c1[q4 * 4], kt_c1[q4 * 4 + 1], kt_c1[q4 * 4 + 2], kt_c1[q4 * 4 + 3]);
+      }
+    }
+    tc::fence_async_smem();
+    cta_sync_tc();
+
+    // ---- P2: Gram MMA (M=128, N=160, K=128) ------------------------------
+    if (tid == 0) {
+      constexpr uint32_t idesc = tc::make_idesc(1, 0, 0, 128, 160);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint64_t da =
+            tc::make_desc(sbase + OFF_AG + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+        const uint64_t db =
+            tc::make_desc(sbase + OFF_BG + (ks >> 2) * 20480 + (ks & 3) * 32, 16, 1024);
+        tc::mma_bf16_ss(tmem + TM_G, da, db, idesc, ks > 0 ? 1u : 0u);
+      }
+      tc::mma_commit(mbar);
+    }
+    ok = cta_wait(mbar, phase, 1);
+    phase ^= 1;
+    if (!ok) break;
+
+    // ---- P3: rows of M_kk (lanes 0..63) and M_qk (lanes 64..127) ---------
+    if (warp < 4) {
+      const int row = warp * 32 + lane;
+      const bool is_q = row >= 64;
+      const int r = row & 63;
+      const int ar = r >> 4;
+      const uint32_t tb = tmem + (static_cast<uint32_t>(warp * 32) << 16) + TM_G;
+      const float br = s_beta[r];
+      float* nmat = reinterpret_cast<float*>(smem + OFF_NMAT);
+#pragma unroll
+      for (int jg = 0; jg < 4; ++jg) {
+        float dg[16], r1[16], r2[16], r3[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) r1[i] = r2[i] = r3[i] = 0.f;
+        tc::tmem_ld16(tb + jg * 16, dg);
+        if (jg == 0) tc::tmem_ld16(tb + 64, r1);
+        if (jg < 2) tc::tmem_ld16(tb + 80 + jg * 16, r2);
+        if (jg < 3) tc::tmem_ld16(tb + 112 + jg * 16, r3);
+        tc::tmem_wait_ld();
+        float out[16];
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+          const int j = jg * 16 + jj;
+          float val = 0.f;
+          if (jg < ar)
+            val = ar == 1 ? r1[jj] : (ar == 2 ? r2[jj] : r3[jj]);
+          else if (jg == ar)
+            val = (is_q ? (j <= r) : (j < r)) ? dg[jj] : 0.f;
+          out[jj] = val;
+        }
+        if (!is_q) {
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) nmat[r * 65 + jg * 16 + jj] = br * out[jj];
+        } else {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            *reinterpret_cast<float4*>(smem + OFF_MQK +
+                                       tc::sw128<4>(r, jg * 16 + q4 * 4, 64)) =
+                make_float4(out[q4 * 4], out[q4 * 4 + 1], out[q4 * 4 + 2], out[q4 * 4 + 3]);
+        }
+      }
+    }
+    tc::fence_async_smem();
+    cta_sync_tc();
+
+    // ---- P4: X = (I + N)^-1 by block forward substitution (16 x 16) ------
+    {
+      const float* N = reinterpret_cast<const float*>(smem + OFF_NMAT);
+      float* X = reinterpret_cast<float*>(smem + OFF_XMAT);
+      float* Y = reinterpret_cast<float*>(smem + OFF_YBUF);
+      if (tid < 64) {
+        const int base = (tid >> 4) * 16, col = tid & 15;
+        float x[16];
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) {
+          float acc = rr == col ? 1.f : 0.f;
+#pragma unroll
+          for (int jj = 0; jj < rr; ++jj) acc -= N[(base + rr) * 65 + base + jj] * x[jj];
+          x[rr] = acc;
+        }
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) X[(base + rr) * 65 + base + col] = x[rr];
+      }
+      __syncthreads();
+      const int rr = tid >> 4, cc = tid & 15;
+      for (int a = 1; a < 4; ++a) {
+        for (int b = 0; b < a; ++b) {
+          float acc = 0.f;
+          for (int c = b; c < a; ++c) {
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj)
+              acc += N[(a * 16 + rr) * 65 + c * 16 + jj] * X[(c * 16 + jj) * 65 + b * 16 + cc];
+          }
+          Y[(b * 16 + rr) * 17 + cc] = acc;
+        }
+        __syncthreads();
+        for (int b = 0; b < a; ++b) {
+          float acc = 0.f;
+#pragma unroll
+          for (int kk = 0; kk < 16; ++kk)
+            acc += X[(a * 16 + rr) * 65 + a * 16 + kk] * Y[(b * 16 + kk) * 17 + cc];
+          X[(a * 16 + rr) * 65 + b * 16 + cc] = -acc;
+        }
+        __syncthreads();
+      }
+      // T = X diag(beta) (lower triangle incl. diagonal) -> bf16 K-major [r][j]
+      {
+        const int r = tid >> 2, j0 = (tid & 3) * 16;
+#pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            const int j = j0 + h8 * 8 + e;
+            const float x0 = j <= r ? X[r * 65 + j] * s_beta[j] : 0.f;
+            const float x1 = j + 1 <= r ? X[r * 65 + j + 1] * s_beta[j + 1] : 0.f;
+            w[e >> 1] = pack_bf16x2(x0, x1);
+          }
+          *reinterpret_cast<uint4*>(smem + OFF_TM + tc::sw128<2>(r, j0 + h8 * 8, 64)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+    tc::fence_async_smem();
+    cta_sync_tc();
+
+    // ---- P5: W^T = (K e^g)^T T^T and U^T = V^T T^T (M=128, N=64, K=64) ----
+    if (tid == 0) {
+      constexpr uint32_t idesc = tc::make_idesc(1, 1, 0, 128, 64);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const uint64_t dw = tc::make_desc(sbase + OFF_BK + ks * 2048, 8192, 1024);
+        const uint64_t du = tc::make_desc(sbase + OFF_VV + ks * 2048, 8192, 1024);
+        const uint64_t dt = tc::make_desc(sbase + OFF_TM + ks * 32, 16, 1024);
+        tc::mma_bf16_ss(tmem + TM_W, dw, dt, idesc, ks > 0 ? 1u : 0u);
+        tc::mma_bf16_ss(tmem + TM_D, du, dt, idesc, ks > 0 ? 1u : 0u);
+      }
+      tc::mma_commit(mbar);
+    }
+    ok = cta_wait(mbar, phase, 2);
+    phase ^= 1;
+    if (!ok) break;
+
+    // ---- P6: -W^T to shared memory; S0 -> bf16; decay of the fp32 state --
+    if (warp < 4) {
+      const int c = warp * 32 + lane;
+      const uint32_t tb = tmem + (static_cast<uint32_t>(warp * 32) << 16) + TM_W;
+#pragma unroll
+      for (int rg = 0; rg < 4; ++rg) {
+        float w[16];
+        tc::tmem_ld16(tb + rg * 16, w);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8) {
+          uint32_t p[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            p[e] = pack_bf16x2(-w[h8 * 8 + 2 * e], -w[h8 * 8 + 2 * e + 1]);
+          *reinterpret_cast<uint4*>(smem + OFF_NW + tc::sw128<2>(c, rg * 16 + h8 * 8, 128)) =
+              make_uint4(p[0], p[1], p[2], p[3]);
+        }
+      }
+    }
+    {
+      const uint32_t tb = tmem + lane_off + TM_S + half * 64;
+#pragma unroll
+      for (int cg = 0; cg < 4; ++cg) {
+        float s[16];
+        tc::tmem_ld16(tb + cg * 16, s);
+        tc::tmem_wait_ld();
+        const int cb = half * 64 + cg * 16;
+#pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8) {
+          uint32_t p[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) p[e] = pack_bf16x2(s[h8 * 8 + 2 * e], s[h8 * 8 + 2 * e + 1]);
+          *reinterpret_cast<uint4*>(smem + OFF_SB + tc::sw128<2>(m, cb + h8 * 8, 128)) =
+              make_uint4(p[0], p[1], p[2], p[3]);
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) s[i] *= s_gamma[cb + i];
+        tc::tmem_st16(tb + cg * 16, s);
+      }
+      tc::tmem_wait_st();
+    }
+    tc::fence_async_smem();
+    cta_sync_tc();
+
+    // ---- P7: D^T += S0b^T (-W^T);  O^T = S0b^T (Q e^g)^T (K = 128) --------
+    if (tid == 0) {
+      constexpr uint32_t id_d = tc::make_idesc(1, 0, 1, 128, 64);
+      constexpr uint32_t id_o = tc::make_idesc(1, 0, 0, 128, 64);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint64_t da =
+            tc::make_desc(sbase + OFF_SB + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+        const uint64_t dn = tc::make_desc(sbase + OFF_NW + ks * 2048, 16384, 1024);
+        const uint64_t dq =
+            tc::make_desc(sbase + OFF_QT + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+        tc::mma_bf16_ss(tmem + TM_D, da, dn, id_d, 1u);
+        tc::mma_bf16_ss(tmem + TM_O, da, dq, id_o, ks > 0 ? 1u : 0u);
+      }
+      tc::mma_commit(mbar);
+    }
+    ok = cta_wait(mbar, phase, 3);
+    phase ^= 1;
+    if (!ok) break;
+
+    // ---- P8: S^T += D^T K~ (tf32, A from TMEM); O^T += D^T M_qk^T ---------
+    if (tid == 0) {
+      constexpr uint32_t id_s = tc::make_idesc(2, 0, 0, 128, 128);
+      constexpr uint32_t id_o = tc::make_idesc(2, 0, 0, 128, 64);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t a_t = tmem + TM_D + ks * 8;
+        const uint64_t dk_ =
+            tc::make_desc(sbase + OFF_KT + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+        const uint64_t dm =
+            tc::make_desc(sbase + OFF_MQK + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+        tc::mma_tf32_ts(tmem + TM_S, a_t, dk_, id_s, 1u);
+        tc::mma_tf32_ts(tmem + TM_O, a_t, dm, id_o, 1u);
+      }
+      tc::mma_commit(mbar);
+    }
+    ok = cta_wait(mbar, phase, 4);
+    phase ^= 1;
+    if (!ok) break;
+
+    // ---- P9: O to HBM (bf16) ---------------------------------------------
+    {
+      const uint32_t tb = tmem + lane_off + TM_O + half * 32;
+#pragma unroll
+      for (int rg = 0; rg < 2; ++rg) {
+        float ov[16];
+        tc::tmem_ld16(tb + rg * 16, ov);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int r = half * 32 + rg * 16 + i;
+          if (r < L) o[((size_t)(t0 + r) * H + head) * DV + m] = __float2bfloat16_rn(ov[i]);
+        }
+      }
+    }
+    cta_sync_tc();
+  }
+
+  if (ok && final_state) {
+    const uint32_t tb = tmem + lane_off + TM_S + half * 64;
+#pragma unroll
+    for (int cg = 0; cg < 4; ++cg) {
+      float s[16];
+      tc::tmem_ld16(tb + cg * 16, s);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int c = half * 64 + cg * 16 + i;
+        final_state[state_off + (size_t)c * DV + m] = s[i];
+      }
+    }
+  }
+  if (!ok) {
+    // A wait gave up: give the outstanding MMAs one more bounded chance to
+    // land before the tensor memory they write is released.
+    if (tid == 0) tc::mbar_wait_bounded(mbar, phase ^ 1, kMaxWaitNs);
+  }
+  cta_sync_tc();
+  if (warp == 0) tc::tmem_dealloc(tmem, 512);
+}
+
+// Longest-first order of the packed sequences (ties by index), so the long
+// chains start first and the short ones fill in behind them.
+__global__ void order_by_length_kernel(const int32_t* __restrict__ cu, int n_seq,
+                                       int32_t* __restrict__ order) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_seq; i += gridDim.x * blockDim.x) {
+    const int li = cu[i + 1] - cu[i];
+    int rank = 0;
+    for (int j = 0; j < n_seq; ++j) {
+      const int lj = cu[j + 1] - cu[j];
+      rank += (lj > li) || (lj == li && j < i);
+    }
+    order[rank] = i;
+  }
+}
+
+__global__ void identity_order_kernel(int n_seq, int32_t* __restrict__ order) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_seq; i += gridDim.x * blockDim.x)
+    order[i] = i;
+}
+
+}  // namespace chunk64
+
+cudaError_t launch_chunk64(const void* q, const void* k, const void* v, const float* la,
+                           const float* beta, const float* s0, const int32_t* cu, int n_seq,
+                           int T, int H, void* o, float* sT, int32_t* order,
+                           cudaStream_t stream) {
+  using namespace chunk64;
+  static bool attr_set = false;
+  if (!attr_set) {
+    const cudaError_t e = cudaFuncSetAttribute(
+        chunk64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  if (cu && order) {
+    const int blocks = (n_seq + 255) / 256;
+    if (n_seq <= 8192)
+      order_by_length_kernel<<<blocks, 256, 0, stream>>>(cu, n_seq, order);
+    else
+      identity_order_kernel<<<blocks, 256, 0, stream>>>(n_seq, order);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  chunk64_kernel<<<(unsigned)((long long)n_seq * H), kThreads, kSmemBytes, stream>>>(
+      (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, la, beta, s0,
+      cu, cu ? order : nullptr, T, H, (__nv_bfloat16*)o, sT);
+  return cudaGetLastError();
+}
+
+}  // namespace kda

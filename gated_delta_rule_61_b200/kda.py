@@ -1,0 +1,176 @@
+"""Python binding of libkda.so (ctypes). Argument marshalling only: every step
+of the recurrence runs in the library's CUDA kernels; there is no fallback.
+
+The C ABI (include/kda.h) takes device pointers; these wrappers take torch
+CUDA tensors, check shapes and dtypes, pass ``data_ptr()`` values and the
+current CUDA stream, and raise ``KdaError`` on a non-OK status.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libkda.so")
+
+# Status codes and dtype codes of include/kda.h.
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_ERR_CUDA, \
+    KDA_ERR_TIMEOUT = range(6)
+KDA_F32, KDA_BF16 = 0, 1
+CHUNK_LOG_ALPHA_MIN = -10.0
+
+EXPORTS = ("kda_status_string", "kda_version", "kda_prefill_workspace_bytes",
+           "kda_prefill", "kda_decode_step", "kda_get_device_status")
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s failed: %s (status %d)" % (what, status_string(status), status))
+
+
+_lib = None
+
+
+def lib():
+    """Load libkda.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError("libkda.so is missing: build it with "
+                           "`python -m gated_delta_rule_61_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, fp, ip, i32p = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p
+    L.kda_status_string.argtypes = [ctypes.c_int]
+    L.kda_status_string.restype = ctypes.c_char_p
+    L.kda_version.argtypes = []
+    L.kda_version.restype = ctypes.c_int
+    L.kda_prefill_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int]
+    L.kda_prefill_workspace_bytes.restype = ctypes.c_size_t
+    L.kda_prefill.argtypes = [vp, vp, vp, fp, fp, fp, i32p, ip, ip, ip, ip, ip, ip,
+                              ctypes.c_int, ctypes.c_int, vp, fp, vp, ctypes.c_size_t, vp]
+    L.kda_prefill.restype = ctypes.c_int
+    L.kda_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, ip, ip, ip, ip, ctypes.c_int, vp, vp]
+    L.kda_decode_step.restype = ctypes.c_int
+    L.kda_get_device_status.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int), vp]
+    L.kda_get_device_status.restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().kda_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    if t.dtype == torch.float32:
+        return KDA_F32
+    raise TypeError("q/k/v must be bfloat16 or float32, got %s" % t.dtype)
+
+
+def _check(t, name, shape, dtype, device):
+    if t.device != device:
+        raise ValueError("%s must be on %s" % (name, device))
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def workspace_bytes(n_seq: int, has_cu_seqlens: bool) -> int:
+    return int(lib().kda_prefill_workspace_bytes(int(n_seq), 1 if has_cu_seqlens else 0))
+
+
+def prefill(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, *, chunk=64,
+            output_final_state=True, o=None, final_state=None, workspace=None, stream=None):
+    """Chunked (chunk=64) or token-recurrent (chunk=0) KDA prefill.
+
+    q, k, log_alpha [B, T, H, dk]; v [B, T, H, dv]; beta [B, T, H];
+    init_state [N, H, dk, dv] or None; cu_seqlens int32 [N+1] (then B = 1).
+    Returns (o [B, T, H, dv] in q's dtype, final_state [N, H, dk, dv] fp32 or
+    None).
+    """
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    dt = q.dtype
+    code = _dtype_code(q)
+    n_seq = B if cu_seqlens is None else cu_seqlens.shape[0] - 1
+    _check(q, "q", (B, T, H, dk), dt, dev)
+    _check(k, "k", (B, T, H, dk), dt, dev)
+    _check(v, "v", (B, T, H, dv), dt, dev)
+    _check(log_alpha, "log_alpha", (B, T, H, dk), torch.float32, dev)
+    _check(beta, "beta", (B, T, H), torch.float32, dev)
+    if init_state is not None:
+        _check(init_state, "init_state", (n_seq, H, dk, dv), torch.float32, dev)
+    if cu_seqlens is not None:
+        if B != 1:
+            raise ValueError("packed sequences (cu_seqlens) need B == 1")
+        _check(cu_seqlens, "cu_seqlens", (n_seq + 1,), torch.int32, dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+    else:
+        _check(o, "o", (B, T, H, dv), dt, dev)
+    if output_final_state and final_state is None:
+        final_state = torch.empty((n_seq, H, dk, dv), dtype=torch.float32, device=dev)
+    elif final_state is not None:
+        _check(final_state, "final_state", (n_seq, H, dk, dv), torch.float32, dev)
+    need = workspace_bytes(n_seq, cu_seqlens is not None) if chunk else 0
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().kda_prefill(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(init_state),
+        _ptr(cu_seqlens), int(n_seq), int(B), int(T), int(H), int(dk), int(dv), code,
+        int(chunk), _ptr(o), _ptr(final_state), _ptr(workspace), ws_bytes, _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_prefill")
+    return o, final_state
+
+
+def decode_step(q, k, v, log_alpha, beta, state, *, o=None, stream=None):
+    """One decode token per sequence; ``state`` [B, H, dk, dv] fp32 is
+    updated in place. Returns o [B, H, dv] in q's dtype."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    code = _dtype_code(q)
+    _check(q, "q", (B, H, dk), dt, dev)
+    _check(k, "k", (B, H, dk), dt, dev)
+    _check(v, "v", (B, H, dv), dt, dev)
+    _check(log_alpha, "log_alpha", (B, H, dk), torch.float32, dev)
+    _check(beta, "beta", (B, H), torch.float32, dev)
+    _check(state, "state", (B, H, dk, dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=dt, device=dev)
+    else:
+        _check(o, "o", (B, H, dv), dt, dev)
+    st = lib().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                               _ptr(state), int(B), int(H), int(dk), int(dv), code, _ptr(o),
+                               _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_decode_step")
+    return o
+
+
+def device_status(reset: bool = True, stream=None):
+    """(status, detail) of the device status word; synchronises the stream."""
+    detail = ctypes.c_int(0)
+    st = lib().kda_get_device_status(1 if reset else 0, ctypes.byref(detail), _stream(stream))
+    return int(st), int(detail.value)

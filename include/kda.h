@@ -1,0 +1,142 @@
+/*
+ * kda.h -- C ABI of libkda.so: the Kimi Delta Attention (KDA) channel-wise
+ * gated delta-rule recurrence on NVIDIA B200 (sm_100a).
+ *
+ * The operation (per sequence and head; state S is dk x dv, fp32):
+ *     S'  = Diag(exp(log_alpha_t)) S        one decay per KEY channel (row)
+ *     r   = S'^T k_t                        value the key reads now
+ *     S   = S' + k_t (beta_t (v_t - r))^T   delta write
+ *     o_t = S^T q_t                         read-out after the write
+ * Sources: "22580: from GPT-2 to Kimi K3, explained" (temp07.ru; English
+ * original at marvinlee.cn), sections "DeltaNet, or Fast Weight Programmers"
+ * (cached forward: read at the key, subtract, write the outer product, read
+ * out with no denominator), "DeltaNet, or Parallelizing Linear Transformers
+ * with Delta Rule" (token loop for prefill and the chunk-wise form),
+ * "Gated Delta Net" (the decay alpha: 1 = pure delta rule, 0 = clear) and
+ * "KDA / Kimi Linear" (a separate decay per channel); the ai-flip.ru KDA
+ * explainer, section on channel-wise gating (a diagonal gate matrix) and on
+ * chunking for tensor cores.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the
+ *     library never allocates, frees or keeps them. Tensors are contiguous
+ *     and row-major in the shapes given below.
+ *   - q and k are used as given (no normalisation, no 1/sqrt(d) scale).
+ *   - log_alpha = log(alpha) <= 0 (fp32). -INFINITY is a full clear. The
+ *     chunked prefill path clamps log_alpha to >= KDA_CHUNK_LOG_ALPHA_MIN
+ *     (alpha >= 4.5e-5) so its within-chunk factorisation stays finite; the
+ *     token-recurrent and decode kernels apply the gate exactly.
+ *   - Work is enqueued on `stream` and runs asynchronously. Argument errors
+ *     are reported synchronously (nothing is launched); launch failures map
+ *     to KDA_ERR_CUDA; a device-side timeout of a bounded wait is recorded in
+ *     a device status word read by kda_get_device_status().
+ *   - Supported head sizes: dk, dv in {64, 128}. The chunked tensor-core
+ *     path needs dk = dv = 128, bf16 inputs and chunk = 64.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, bad cu_seqlens shape */
+    KDA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (head size, chunk) */
+    KDA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required   */
+    KDA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed         */
+    KDA_ERR_TIMEOUT = 5        /* a bounded device-side wait gave up           */
+} kda_status;
+
+typedef enum {
+    KDA_F32 = 0,               /* q, k, v and o are fp32                       */
+    KDA_BF16 = 1               /* q, k, v and o are bf16                       */
+} kda_dtype;
+
+/* Lower bound applied to log_alpha by the chunked prefill path. */
+#define KDA_CHUNK_LOG_ALPHA_MIN (-10.0f)
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *kda_status_string(kda_status status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int kda_version(void);
+
+/*
+ * Bytes of workspace kda_prefill needs for n_seq packed sequences (the
+ * longest-first work order of the variable-length driver). 0 when
+ * cu_seqlens will be NULL. Never fails; n_seq < 0 is treated as 0.
+ */
+size_t kda_prefill_workspace_bytes(int n_seq, int has_cu_seqlens);
+
+/*
+ * kda_prefill -- run the recurrence over whole sequences (prefill), with an
+ * optional cached initial state, returning every output and the final state.
+ *
+ * Dense batch (cu_seqlens == NULL): B sequences of T tokens.
+ *   q, k       [B, T, H, dk]  dtype          v, o   [B, T, H, dv]  dtype
+ *   log_alpha  [B, T, H, dk]  fp32           beta   [B, T, H]      fp32
+ *   init_state [B, H, dk, dv] fp32 or NULL (zeros)
+ *   final_state[B, H, dk, dv] fp32 or NULL (not written)
+ *   n_seq must be B (or 0, meaning B).
+ * Packed variable length (cu_seqlens != NULL, a DEVICE int32 array of
+ * n_seq + 1 offsets, cu[0] = 0, non-decreasing, cu[n_seq] = T): B must be 1,
+ *   the token tensors are [1, T, H, *], sequence i owns tokens
+ *   [cu[i], cu[i+1]) and starts from init_state[i] (or zeros), and
+ *   init_state / final_state are [n_seq, H, dk, dv]. A zero-length sequence
+ *   copies its initial state to its final state. The offsets are read on the
+ *   device only; offsets that break the rules above give undefined output but
+ *   never an out-of-bounds access (each sequence is clamped to [0, T)).
+ * chunk: 0 selects the token-recurrent kernel (fp32 state in registers, any
+ *   supported head size and dtype, exact gate). 64 selects the chunked
+ *   tensor-core kernel (tcgen05 MMAs with TMEM accumulators; bf16 inputs,
+ *   dk = dv = 128). With dtype KDA_F32 the recurrent kernel always runs.
+ * final_state may alias init_state (each chain reads its initial state
+ *   before writing its final one). o must not alias any input.
+ * workspace: at least kda_prefill_workspace_bytes(n_seq, cu_seqlens != NULL)
+ *   bytes of device memory, 256-byte aligned; may be NULL when that is 0.
+ */
+kda_status kda_prefill(const void *q, const void *k, const void *v,
+                       const float *log_alpha, const float *beta,
+                       const float *init_state, const int32_t *cu_seqlens,
+                       int n_seq, int B, int T, int H, int dk, int dv,
+                       kda_dtype dtype, int chunk,
+                       void *o, float *final_state,
+                       void *workspace, size_t workspace_bytes,
+                       cudaStream_t stream);
+
+/*
+ * kda_decode_step -- one token per sequence against a cached state, updated
+ * in place (the pages' decode call: the same forward with one token and the
+ * cache from the previous call).
+ *   q, k       [B, H, dk]  dtype            v, o  [B, H, dv]  dtype
+ *   log_alpha  [B, H, dk]  fp32             beta  [B, H]      fp32
+ *   state      [B, H, dk, dv] fp32, read and overwritten with the new state
+ * The kernel is HBM-bound: each head's state is read once and written once.
+ */
+kda_status kda_decode_step(const void *q, const void *k, const void *v,
+                           const float *log_alpha, const float *beta,
+                           float *state, int B, int H, int dk, int dv,
+                           kda_dtype dtype, void *o, cudaStream_t stream);
+
+/*
+ * kda_get_device_status -- synchronise `stream` and return the sticky device
+ * status word of the current device: KDA_OK, or KDA_ERR_TIMEOUT when a
+ * bounded wait inside a kernel gave up since the last reset (the kernel then
+ * stopped its chain early, released its tensor memory and left its outputs
+ * incomplete). If `reset` is non-zero the word is cleared after reading.
+ * `detail` (may be NULL) receives an implementation-defined code naming the
+ * wait that gave up (0 when none did).
+ */
+kda_status kda_get_device_status(int reset, int *detail, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

@@ -1,0 +1,120 @@
+"""The C-ABI library loads, exports every entry point include/kda.h declares,
+and rejects bad arguments synchronously (no GPU needed: argument checks run
+before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from gated_delta_rule_61_b200 import kda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+FAKE = ctypes.c_void_p(0x10000)   # never dereferenced: checks fail first
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert set(_declared()) == set(kda.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = kda.lib()
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_version():
+    for code in range(6):
+        assert kda.status_string(code)
+    assert kda.status_string(99) == "unknown status"
+    assert kda.lib().kda_version() >= 100
+
+
+def test_workspace_query():
+    assert kda.workspace_bytes(64, False) == 0
+    assert kda.workspace_bytes(0, True) == 0
+    assert kda.workspace_bytes(1, True) == 256
+    assert kda.workspace_bytes(64, True) == 256
+    assert kda.workspace_bytes(65, True) == 512
+
+
+def _prefill(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, s0=None, cu=None, n_seq=0, B=1, T=64,
+             H=2, dk=128, dv=128, dtype=kda.KDA_BF16, chunk=64, o=FAKE, sT=None, ws=None,
+             ws_bytes=0, stream=None)
+    a.update(kw)
+    return kda.lib().kda_prefill(a["q"], a["k"], a["v"], a["la"], a["beta"], a["s0"], a["cu"],
+                                 a["n_seq"], a["B"], a["T"], a["H"], a["dk"], a["dv"],
+                                 a["dtype"], a["chunk"], a["o"], a["sT"], a["ws"],
+                                 a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(H=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(B=-1), kda.KDA_ERR_INVALID_ARG),
+    (dict(T=-5), kda.KDA_ERR_INVALID_ARG),
+    (dict(dtype=7), kda.KDA_ERR_INVALID_ARG),
+    (dict(q=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(beta=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(o=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(n_seq=3, B=2), kda.KDA_ERR_INVALID_ARG),
+    (dict(cu=FAKE, B=2, n_seq=2), kda.KDA_ERR_INVALID_ARG),
+    (dict(dk=96), kda.KDA_ERR_UNSUPPORTED),
+    (dict(dv=32), kda.KDA_ERR_UNSUPPORTED),
+    (dict(chunk=32), kda.KDA_ERR_UNSUPPORTED),
+    (dict(dk=64, dv=64), kda.KDA_ERR_UNSUPPORTED),        # chunked path is dk = dv = 128
+    (dict(cu=FAKE, n_seq=4), kda.KDA_ERR_WORKSPACE),       # varlen needs its workspace
+    (dict(cu=FAKE, n_seq=4, ws=FAKE, ws_bytes=16), kda.KDA_ERR_WORKSPACE),
+    (dict(cu=FAKE, n_seq=4, ws=ctypes.c_void_p(0x10004), ws_bytes=256), kda.KDA_ERR_WORKSPACE),
+])
+def test_prefill_rejects_bad_arguments(kw, status):
+    assert _prefill(**kw) == status
+
+
+def test_prefill_empty_is_ok_without_touching_memory():
+    assert _prefill(B=0, T=0, q=None, k=None, v=None, la=None, beta=None, o=None) == kda.KDA_OK
+
+
+def _decode(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, state=FAKE, B=2, H=2, dk=128, dv=128,
+             dtype=kda.KDA_BF16, o=FAKE, stream=None)
+    a.update(kw)
+    return kda.lib().kda_decode_step(a["q"], a["k"], a["v"], a["la"], a["beta"], a["state"],
+                                     a["B"], a["H"], a["dk"], a["dv"], a["dtype"], a["o"],
+                                     a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(H=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(B=-2), kda.KDA_ERR_INVALID_ARG),
+    (dict(dtype=3), kda.KDA_ERR_INVALID_ARG),
+    (dict(state=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(o=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(state=ctypes.c_void_p(0x10004)), kda.KDA_ERR_INVALID_ARG),   # 16-byte alignment
+    (dict(dk=100), kda.KDA_ERR_UNSUPPORTED),
+    (dict(B=0), kda.KDA_OK),
+])
+def test_decode_rejects_bad_arguments(kw, status):
+    assert _decode(**kw) == status
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device error path")
+def test_launch_without_device_reports_cuda_error():
+    assert _decode() == kda.KDA_ERR_CUDA
+    assert _prefill(chunk=0) == kda.KDA_ERR_CUDA
+
+
+def test_python_wrapper_checks_shapes_before_the_library():
+    q = torch.zeros(1, 4, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises((ValueError, TypeError)):
+        kda.prefill(q, q, q, torch.zeros(1, 4, 2, 64), torch.zeros(1, 4, 2))
+    with pytest.raises(TypeError):
+        kda.prefill(q.half(), q.half(), q.half(), torch.zeros(1, 4, 2, 128), torch.zeros(1, 4, 2))
