@@ -1,0 +1,375 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA hot path on B200.
+
+Step = one chunked prefill (tensor-core kernel) of the mid-size prefill
+workload: B=4, T=8192, H=16, dk=dv=128, bf16 q/k/v, fp32 log_alpha and beta,
+N(0, 0.1^2) fp32 initial state, chunk C=64 (inputs resident in HBM).
+Metric: tokens/s (positions B*T per second, all heads). The same JSON line
+carries the decode-step workload (B=256 sequences, H=32, d=128, fp32 state
+[256,32,128,128] updated in place, bf16 inputs, fresh inputs every step) as
+state-update GB/s, each with its roofline fraction.
+
+  python bench.py [--gpus N --steps K --warmup W]        # this library
+  python bench.py --impl reference [...]                 # the fp64 CPU oracle
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own copy of
+the workload (independent sequences: no data-path collective); the time is
+the max over ranks and the value counts the tokens of all ranks.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KDA prefill tokens/s & decode state GB/s (fraction of B200 roofline), 1 GPU"
+PREFILL = dict(B=4, T=8192, H=16, dk=128, dv=128, chunk=64, init_std=0.1)
+DECODE = dict(B=256, H=32, dk=128, dv=128, std=0.05)
+BYTES_PER_HEAD_TOKEN = 3 * 256 + 512 + 4 + 256        # q,k,v + log_alpha + beta + o
+FLOPS_PER_HEAD_TOKEN = 6 * 128 * 128 + 2 * 64 * (3 * 128 + 2 * 128)   # dense tiles, C = 64
+PROFILE = os.path.join(ROOT, "profiles", "chunk64_prefill_b4_t8192_h16.txt")
+KERNEL_SRC = os.path.join(ROOT, "gated_delta_rule_61_b200", "csrc", "kda_chunk.cu")
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def kernel_traffic():
+    """dram bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    try:
+        text = open(PROFILE).read()
+        src_hash = hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()[:16]
+        fields = dict(line.split(":", 1) for line in text.splitlines() if ":" in line)
+        if fields.get("kernel_source_sha256_16", "").strip() != src_hash:
+            return None
+        return int(fields["dram_bytes_per_launch"].strip())
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 50 ms during the timed regions."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.p is not None:
+            self.p.terminate()
+            try:
+                self.p.wait(timeout=5)
+            except Exception:
+                self.p.kill()
+
+    def summary(self):
+        try:
+            self.f.seek(0)
+            rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.strip()]
+        except Exception:
+            rows = []
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if "Active" in v
+                          and "Not" not in v})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def cpu_oracle_prefill(budget_s=12.0, seed=0):
+    """Time the fp64 oracle on a bounded sample of the prefill workload: all
+    B*H chains over their first `n_tok` tokens, n_tok sized to about
+    `budget_s` seconds from a short calibration run."""
+    import torch
+    import oracle
+    from gated_delta_rule_61_b200.inputs import prefill_inputs
+    P = PREFILL
+    cores = oracle.default_threads()
+
+    def run(n_tok):
+        inp = prefill_inputs(P["B"], n_tok, P["H"], P["dk"], P["dv"], dtype=torch.bfloat16,
+                             seed=seed, init_std=P["init_std"])
+        t0 = time.perf_counter()
+        oracle.kda_forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                           init_state=inp["init_state"], n_threads=cores)
+        return time.perf_counter() - t0
+
+    cal = 32
+    dt = run(cal)
+    n_tok = int(max(cal, min(P["T"], cal * budget_s / max(dt, 1e-6))))
+    dt = run(n_tok)
+    tok_s = P["B"] * n_tok / dt
+    return tok_s, cores, n_tok, dt
+
+
+def bench_reference(args):
+    world, rank, _ = (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+                      0)
+    if rank != 0:
+        return
+    times, n_toks, cores = [], [], None
+    for i in range(args.warmup + args.steps):
+        tok_s, cores, n_tok, dt = cpu_oracle_prefill(budget_s=args.ref_budget, seed=i)
+        if i >= args.warmup:
+            times.append(tok_s)
+            n_toks.append(n_tok)
+    value = statistics.median(times)
+    P = PREFILL
+    sample = ("all %d (batch, head) chains, first %d of %d tokens, fp64 oracle"
+              % (P["B"] * P["H"], min(n_toks), P["T"]))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * P["B"] * P["T"] / value, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "KDA prefill B=4 T=8192 H=16 dk=dv=128 bf16 inputs, C=64",
+                       "global_batch": P["B"], "seq_len": P["T"], "heads": P["H"],
+                       "parallelism": "replicas"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def bench_ours(args):
+    import torch
+    from gated_delta_rule_61_b200 import kda
+    from gated_delta_rule_61_b200.inputs import decode_inputs, decode_state, prefill_inputs
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    P, D = PREFILL, DECODE
+    hbm, bf16_tf, peak_kind = peaks()
+
+    # ---------------- prefill (the headline step) ----------------
+    inp = prefill_inputs(P["B"], P["T"], P["H"], P["dk"], P["dv"], dtype=torch.bfloat16,
+                         seed=1000 + rank, init_std=P["init_std"], device=dev)
+    o = torch.empty_like(inp["v"])
+    fs = torch.empty_like(inp["init_state"])
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        kda.prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                    init_state=inp["init_state"], chunk=P["chunk"], o=o, final_state=fs,
+                    stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    barrier(world)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    clk = ClockSampler(local).__enter__()
+    if True:
+        barrier(world)
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        t_end.record(stream)
+        barrier(world)
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
+    kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    ms_per_step = total_ms / args.steps
+    tokens = P["B"] * P["T"]
+    value = world * tokens / (ms_per_step * 1e-3)
+    head_tokens = tokens * P["H"]
+    state_bytes = 2 * P["B"] * P["H"] * P["dk"] * P["dv"] * 4
+    alg_bytes = head_tokens * BYTES_PER_HEAD_TOKEN + state_bytes
+    achieved_gbs = alg_bytes / (kernel_ms * 1e-3) / 1e9
+    traffic = kernel_traffic()
+    tflops = head_tokens * FLOPS_PER_HEAD_TOKEN / (kernel_ms * 1e-3) / 1e12
+    st, detail = kda.device_status()
+    if st != kda.KDA_OK:
+        raise RuntimeError("device status %d (detail %d) after the timed region" % (st, detail))
+
+    # ---------------- decode (second half of the metric) ----------------
+    dec = None
+    if not args.no_decode:
+        S = decode_state(D["B"], D["H"], D["dk"], D["dv"], std=D["std"], seed=7 + rank,
+                         device=dev)
+        n_in = min(args.decode_steps, 1000)
+        steps_in = [decode_inputs(D["B"], D["H"], D["dk"], D["dv"], dtype=torch.bfloat16,
+                                  seed=7 + rank, step=i, device=dev) for i in range(n_in)]
+        od = torch.empty(D["B"], D["H"], D["dv"], dtype=torch.bfloat16, device=dev)
+
+        def dstep(i):
+            d = steps_in[i % n_in]
+            kda.decode_step(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S, o=od,
+                            stream=stream)
+
+        for i in range(args.warmup):
+            dstep(i)
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(args.decode_steps):
+            dstep(i)
+        b.record(stream)
+        barrier(world)
+        dms = max_over_ranks(a.elapsed_time(b), world) / args.decode_steps
+        per_step_bytes = D["B"] * D["H"] * (2 * D["dk"] * D["dv"] * 4 + BYTES_PER_HEAD_TOKEN)
+        gbs = world * per_step_bytes / (dms * 1e-3) / 1e9
+        dec = {"value": gbs, "unit": "GB/s", "ms_per_step": dms, "steps": args.decode_steps,
+               "tokens_per_s": world * D["B"] / (dms * 1e-3),
+               "workload": "KDA decode B=256 H=32 dk=dv=128, fp32 state in place, bf16 inputs",
+               "roofline": {"bound": "hbm", "achieved": gbs / world, "peak": hbm,
+                            "unit": "GB/s", "frac": gbs / world / hbm, "traffic": None,
+                            "peak_kind": peak_kind}}
+        del steps_in, S
+    clk.__exit__(None, None, None)
+
+    # ---------------- end to end through the public API (host buffers) ----------------
+    e2e = None
+    if not args.no_e2e:
+        host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in inp.items()}
+        o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        s_h = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+        d2h = o_h.numel() * o_h.element_size() + s_h.numel() * s_h.element_size()
+
+        def e2e_step():
+            g = {k: (v.to(dev, non_blocking=True) if v is not None else None)
+                 for k, v in host.items()}
+            oo, ss = kda.prefill(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"],
+                                 init_state=g["init_state"], chunk=P["chunk"], stream=stream)
+            o_h.copy_(oo, non_blocking=True)
+            s_h.copy_(ss, non_blocking=True)
+
+        e2e_step()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(1, min(args.steps, 5))
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        barrier(world)
+        ems = max_over_ranks(a.elapsed_time(b), world) / n_e2e
+        e2e = {"value": world * tokens / (ems * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tok_s, cores, n_tok, dt = cpu_oracle_prefill(budget_s=args.cpu_budget)
+        cpu = {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": "all %d (batch, head) chains, first %d of %d tokens (%.1f s)"
+                         % (P["B"] * P["H"], n_tok, P["T"], dt)}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": "KDA prefill B=4 T=8192 H=16 dk=dv=128 bf16 q/k/v, fp32 "
+                                   "gates and state, chunk C=64 (per GPU)",
+                       "global_batch": P["B"] * world, "seq_len": P["T"], "heads": P["H"],
+                       "parallelism": "replicas (dp%d)" % world,
+                       "l2": "inputs larger than L2 (%.0f MB read per step)" % (alg_bytes / 1e6)},
+            "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm,
+                         "unit": "GB/s", "frac": achieved_gbs / hbm, "traffic": traffic,
+                         "peak_kind": peak_kind, "kernel_ms": kernel_ms,
+                         "tensor": {"achieved_tflops": tflops, "peak_tflops": bf16_tf,
+                                    "frac": tflops / bf16_tf}},
+            "decode": dec, "e2e": e2e, "cpu_baseline": cpu,
+            "gpu_launches": args.steps, "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=60)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--ref-budget", type=float, default=8.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        bench_reference(args)
+    else:
+        bench_ours(args)
+
+
+if __name__ == "__main__":
+    main()

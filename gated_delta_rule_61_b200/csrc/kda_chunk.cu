@@ -68,9 +68,10 @@ constexpr uint32_t OFF_AG = 114688;    // Gram A bf16 K-major [128][c]        32
 constexpr uint32_t OFF_MQK = OFF_AG;           // after the Gram MMA: M_qk fp32 K-major [r][j]
 constexpr uint32_t OFF_TM = OFF_AG + 16384;    // T bf16 K-major [r][j]
 constexpr uint32_t OFF_BG = 147456;    // Gram B bf16 K-major [160][c]        40960
-constexpr uint32_t OFF_NMAT = OFF_BG;          // after the Gram MMA: diag(beta) M_kk, fp32 [64][65]
-constexpr uint32_t OFF_XMAT = OFF_BG + 16640;  // X, fp32 [64][65]
-constexpr uint32_t OFF_YBUF = OFF_BG + 33280;  // block products, fp32 [3][16][17]
+constexpr int kLd = 68;                        // row stride (floats) of the solve's matrices
+constexpr uint32_t OFF_NMAT = OFF_BG;          // after the Gram MMA: diag(beta) M_kk, fp32 [64][68]
+constexpr uint32_t OFF_XMAT = OFF_BG + 17408;  // X, fp32 [64][68]
+constexpr uint32_t OFF_ZBUF = OFF_BG + 34816;  // block products, fp32 [32][34]
 constexpr uint32_t OFF_NW = OFF_BG;            // after the solve: -W^T bf16 MN-major [c][r]
 constexpr uint32_t OFF_MISC = 188416;
 constexpr uint32_t MISC_GAMMA = 0, MISC_BETA = 512, MISC_TOT = 768, MISC_MID = 2816,
@@ -100,6 +101,91 @@ __device__ __forceinline__ void cta_sync_tc() {
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
+}
+
+// X = (I + N)^-1 for the strictly lower 64 x 64 matrix N (row stride kLd),
+// as a recursive 2 x 2 block inverse: for a unit lower block matrix
+// [[A, 0], [C, D]] the inverse is [[A^-1, 0], [-D^-1 C A^-1, D^-1]].
+// Level 1 inverts the four 16 x 16 diagonal blocks by forward substitution,
+// level 2 fills the two 16 x 16 blocks below them, level 3 the 32 x 32 block.
+// All 256 threads take part; entries above the diagonal are never read.
+__device__ __forceinline__ void invert_diag_block(const float* N, float* X, int t) {
+  const int base = (t >> 4) * 16, col = t & 15;
+  float x[16];
+#pragma unroll
+  for (int rr = 0; rr < 16; ++rr) {
+    const float* nr = N + (base + rr) * kLd + base;
+    float a0 = rr == col ? 1.f : 0.f, a1 = 0.f;
+#pragma unroll
+    for (int jj = 0; jj + 1 < rr; jj += 2) {
+      a0 -= nr[jj] * x[jj];
+      a1 -= nr[jj + 1] * x[jj + 1];
+    }
+    if (rr & 1) a0 -= nr[rr - 1] * x[rr - 1];
+    x[rr] = a0 + a1;
+  }
+#pragma unroll
+  for (int rr = 0; rr < 16; ++rr) X[(base + rr) * kLd + base + col] = x[rr];
+}
+
+__device__ __forceinline__ void invert_unit_lower64(const float* N, float* X, float* Z, int t) {
+  if (t < 64) invert_diag_block(N, X, t);
+  __syncthreads();
+  // Level 2: blocks (1,0) and (3,2): Z_p = N_{b a} X_{a a}, X_{b a} = -X_{b b} Z_p.
+  {
+    const int p = t >> 7, rr = (t >> 3) & 15, cc = (t & 7) * 2;
+    const int a = 2 * p * 16, b = a + 16;
+    float z0 = 0.f, z1 = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      const float nv = N[(b + rr) * kLd + a + kk];
+      const float2 xv = *reinterpret_cast<const float2*>(X + (a + kk) * kLd + a + cc);
+      z0 += nv * xv.x;
+      z1 += nv * xv.y;
+    }
+    *reinterpret_cast<float2*>(Z + (p * 16 + rr) * 34 + cc) = make_float2(z0, z1);
+    __syncthreads();
+    float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      const float xv = X[(b + rr) * kLd + b + kk];
+      const float2 zv = *reinterpret_cast<const float2*>(Z + (p * 16 + kk) * 34 + cc);
+      x0 += xv * zv.x;
+      x1 += xv * zv.y;
+    }
+    *reinterpret_cast<float2*>(X + (b + rr) * kLd + a + cc) = make_float2(-x0, -x1);
+    __syncthreads();
+  }
+  // Level 3: Z = N[32:64, 0:32] X[0:32, 0:32];  X[32:64, 0:32] = -X[32:64, 32:64] Z.
+  {
+    const int r2 = (t >> 4) * 2, c2 = (t & 15) * 2;
+    float z00 = 0.f, z01 = 0.f, z10 = 0.f, z11 = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < 32; ++kk) {
+      const float n0 = N[(32 + r2) * kLd + kk], n1 = N[(33 + r2) * kLd + kk];
+      const float2 xv = *reinterpret_cast<const float2*>(X + kk * kLd + c2);
+      const bool live = kk >= c2;  // X[0:32,0:32] is lower triangular
+      const float x0 = live ? xv.x : 0.f, x1 = kk >= c2 + 1 ? xv.y : 0.f;
+      z00 += n0 * x0; z01 += n0 * x1;
+      z10 += n1 * x0; z11 += n1 * x1;
+    }
+    *reinterpret_cast<float2*>(Z + r2 * 34 + c2) = make_float2(z00, z01);
+    *reinterpret_cast<float2*>(Z + (r2 + 1) * 34 + c2) = make_float2(z10, z11);
+    __syncthreads();
+    float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < 32; ++kk) {
+      const bool l0 = kk <= r2, l1 = kk <= r2 + 1;  // X[32:64,32:64] is lower triangular
+      const float d0 = l0 ? X[(32 + r2) * kLd + 32 + kk] : 0.f;
+      const float d1 = l1 ? X[(33 + r2) * kLd + 32 + kk] : 0.f;
+      const float2 zv = *reinterpret_cast<const float2*>(Z + kk * 34 + c2);
+      x00 += d0 * zv.x; x01 += d0 * zv.y;
+      x10 += d1 * zv.x; x11 += d1 * zv.y;
+    }
+    *reinterpret_cast<float2*>(X + (32 + r2) * kLd + c2) = make_float2(-x00, -x01);
+    *reinterpret_cast<float2*>(X + (33 + r2) * kLd + c2) = make_float2(-x10, -x11);
+    __syncthreads();
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -173,18 +259,34 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     const int L = (int)((t_end - t0) < C ? (t_end - t0) : C);
 
     // ---- P1: cumulative gates and operand tiles --------------------------
+    // Every global load of this thread's 16 rows is issued before any use,
+    // so the rows' latencies overlap (the chunk was prefetched into L2 while
+    // the previous chunk ran).
     float g0[16], g1[16];
+    uint32_t kr[16], qr[16], vr[16];
+    float bt[16];
     {
-      float run0 = 0.f, run1 = 0.f;
+      float2 lr[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int r = sub * 16 + i;
-        float2 l = make_float2(0.f, 0.f);
-        if (r < L)
-          l = __ldg(reinterpret_cast<const float2*>(
-              log_alpha + ((size_t)(t0 + r) * H + head) * DK + c0));
-        run0 += fmaxf(l.x, kLogAlphaMin);
-        run1 += fmaxf(l.y, kLogAlphaMin);
+        lr[i] = make_float2(0.f, 0.f);
+        kr[i] = qr[i] = vr[i] = 0u;
+        bt[i] = 0.f;
+        if (r < L) {
+          const size_t tok = (size_t)(t0 + r) * H + head;
+          lr[i] = __ldg(reinterpret_cast<const float2*>(log_alpha + tok * DK + c0));
+          kr[i] = __ldg(reinterpret_cast<const unsigned int*>(k + tok * DK + c0));
+          qr[i] = __ldg(reinterpret_cast<const unsigned int*>(q + tok * DK + c0));
+          vr[i] = __ldg(reinterpret_cast<const unsigned int*>(v + tok * DV + c0));
+          bt[i] = __ldg(beta + tok);
+        }
+      }
+      float run0 = 0.f, run1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        run0 += fmaxf(lr[i].x, kLogAlphaMin);
+        run1 += fmaxf(lr[i].y, kLogAlphaMin);
         g0[i] = run0;
         g1[i] = run1;
       }
@@ -226,47 +328,43 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         rho1[ap] = ap > sub ? expf(s_mid[ap * 128 + c0 + 1] - m1) : 0.f;
       }
       float kt_c0[16], kt_c1[16];
+      // Swizzled byte offsets of this thread's rows (r = 16 sub + i): (r & 7) = (i & 7)
+      // and (r >> 3) = 2 sub + (i >> 3), so only (chunk ^ (i & 7)) varies at run time.
+      const int xr = (c0 & 63) >> 3;
+      const uint32_t colb = (uint32_t)((c0 & 7) * 2) + (uint32_t)sub * 2048u;
+      const uint32_t sl = (uint32_t)(c0 >> 6);
+      uint8_t* const pAGk = smem + OFF_AG + sl * 16384u + colb;
+      uint8_t* const pBGe = smem + OFF_BG + sl * 20480u + colb;
+      uint8_t* const pQT = smem + OFF_QT + sl * 8192u + colb;
+      uint8_t* const pBK = smem + OFF_BK + sl * 8192u + colb;
+      uint8_t* const pVV = smem + OFF_VV + sl * 8192u + colb;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int r = sub * 16 + i;
-        float k0 = 0.f, k1 = 0.f, q0 = 0.f, q1 = 0.f, v0 = 0.f, v1 = 0.f, bt = 0.f;
-        if (r < L) {
-          const size_t tok = (size_t)(t0 + r) * H + head;
-          const float2 kk = __bfloat1622float2(
-              *reinterpret_cast<const __nv_bfloat162*>(k + tok * DK + c0));
-          const float2 qq = __bfloat1622float2(
-              *reinterpret_cast<const __nv_bfloat162*>(q + tok * DK + c0));
-          const float2 vv = __bfloat1622float2(
-              *reinterpret_cast<const __nv_bfloat162*>(v + tok * DV + c0));
-          k0 = kk.x; k1 = kk.y; q0 = qq.x; q1 = qq.y; v0 = vv.x; v1 = vv.y;
-          bt = __ldg(beta + tok);
-        }
-        if (pr == 0) s_beta[r] = bt;
+        const uint32_t ro = (uint32_t)((i >> 3) * 1024 + (i & 7) * 128) +
+                            ((uint32_t)(xr ^ (i & 7)) << 4);
+        // bf16 pairs widen exactly: low half << 16, high half masked.
+        const float k0 = __uint_as_float(kr[i] << 16), k1 = __uint_as_float(kr[i] & 0xffff0000u);
+        const float q0 = __uint_as_float(qr[i] << 16), q1 = __uint_as_float(qr[i] & 0xffff0000u);
+        if (pr == 0) s_beta[r] = bt[i];
         const float f0 = __expf(g0[i] - m0), f1 = __expf(g1[i] - m1);
         const float fi0 = __expf(m0 - g0[i]), fi1 = __expf(m1 - g1[i]);
-        *reinterpret_cast<uint32_t*>(smem + OFF_AG + tc::sw128<2>(r, c0, 128)) =
-            pack_bf16x2(k0 * f0, k1 * f1);
-        *reinterpret_cast<uint32_t*>(smem + OFF_AG + tc::sw128<2>(64 + r, c0, 128)) =
-            pack_bf16x2(q0 * f0, q1 * f1);
+        *reinterpret_cast<uint32_t*>(pAGk + ro) = pack_bf16x2(k0 * f0, k1 * f1);
+        *reinterpret_cast<uint32_t*>(pAGk + ro + 8192) = pack_bf16x2(q0 * f0, q1 * f1);
         const float e0 = k0 * fi0, e1 = k1 * fi1;
-        *reinterpret_cast<uint32_t*>(smem + OFF_BG + tc::sw128<2>(r, c0, 160)) =
-            pack_bf16x2(e0, e1);
+        *reinterpret_cast<uint32_t*>(pBGe + ro) = pack_bf16x2(e0, e1);
         if (sub < 1)
-          *reinterpret_cast<uint32_t*>(smem + OFF_BG + tc::sw128<2>(64 + r, c0, 160)) =
-              pack_bf16x2(e0 * rho0[1], e1 * rho1[1]);
+          *reinterpret_cast<uint32_t*>(pBGe + ro + 8192) = pack_bf16x2(e0 * rho0[1], e1 * rho1[1]);
         if (sub < 2)
-          *reinterpret_cast<uint32_t*>(smem + OFF_BG + tc::sw128<2>(80 + r, c0, 160)) =
+          *reinterpret_cast<uint32_t*>(pBGe + ro + 10240) =
               pack_bf16x2(e0 * rho0[2], e1 * rho1[2]);
         if (sub < 3)
-          *reinterpret_cast<uint32_t*>(smem + OFF_BG + tc::sw128<2>(112 + r, c0, 160)) =
+          *reinterpret_cast<uint32_t*>(pBGe + ro + 14336) =
               pack_bf16x2(e0 * rho0[3], e1 * rho1[3]);
         const float eg0 = f0 * em0, eg1 = f1 * em1;
-        *reinterpret_cast<uint32_t*>(smem + OFF_QT + tc::sw128<2>(r, c0, 64)) =
-            pack_bf16x2(q0 * eg0, q1 * eg1);
-        *reinterpret_cast<uint32_t*>(smem + OFF_BK + tc::sw128<2>(r, c0, 64)) =
-            pack_bf16x2(k0 * eg0, k1 * eg1);
-        *reinterpret_cast<uint32_t*>(smem + OFF_VV + tc::sw128<2>(r, c0, 64)) =
-            pack_bf16x2(v0, v1);
+        *reinterpret_cast<uint32_t*>(pQT + ro) = pack_bf16x2(q0 * eg0, q1 * eg1);
+        *reinterpret_cast<uint32_t*>(pBK + ro) = pack_bf16x2(k0 * eg0, k1 * eg1);
+        *reinterpret_cast<uint32_t*>(pVV + ro) = vr[i];
         kt_c0[i] = e0 * kt0;
         kt_c1[i] = e1 * kt1;
       }
@@ -296,50 +394,84 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       }
       tc::mma_commit(mbar);
     }
+    if (n + 1 < n_chunks) {  // warm L2 with the next chunk's rows
+      const long long t1 = t0 + C;
+      const int row = tid >> 2, part = tid & 3;
+      if (t1 + row < t_end) {
+        const size_t tok = (size_t)(t1 + row) * H + head;
+        if (part == 0) {
+          tc::prefetch_l2(q + tok * DK);
+          tc::prefetch_l2(q + tok * DK + 64);
+        } else if (part == 1) {
+          tc::prefetch_l2(k + tok * DK);
+          tc::prefetch_l2(k + tok * DK + 64);
+        } else if (part == 2) {
+          tc::prefetch_l2(v + tok * DV);
+          tc::prefetch_l2(v + tok * DV + 64);
+          tc::prefetch_l2(beta + tok);
+        } else {
+#pragma unroll
+          for (int l = 0; l < 4; ++l) tc::prefetch_l2(log_alpha + tok * DK + 32 * l);
+        }
+      }
+    }
     ok = cta_wait(mbar, phase, 1);
     phase ^= 1;
     if (!ok) break;
 
     // ---- P3: rows of M_kk (lanes 0..63) and M_qk (lanes 64..127) ---------
-    if (warp < 4) {
-      const int row = warp * 32 + lane;
+    // Warp pair (quad, half): half 0 assembles columns j < 32, half 1 j >= 32.
+    {
+      const int row = quad * 32 + lane;
       const bool is_q = row >= 64;
-      const int r = row & 63;
-      const int ar = r >> 4;
-      const uint32_t tb = tmem + (static_cast<uint32_t>(warp * 32) << 16) + TM_G;
+      const int r = row & 63, ar = r >> 4;
+      const uint32_t tb = tmem + lane_off + TM_G;
       const float br = s_beta[r];
       float* nmat = reinterpret_cast<float*>(smem + OFF_NMAT);
+      float out[32];
+      if (half == 0) {
+        float dg[32], r1[16], r2[32], r3[32];
+        tc::tmem_ld32(tb + 0, dg);
+        tc::tmem_ld16(tb + 64, r1);
+        tc::tmem_ld32(tb + 80, r2);
+        tc::tmem_ld32(tb + 112, r3);
 #pragma unroll
-      for (int jg = 0; jg < 4; ++jg) {
-        float dg[16], r1[16], r2[16], r3[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) r1[i] = r2[i] = r3[i] = 0.f;
-        tc::tmem_ld16(tb + jg * 16, dg);
-        if (jg == 0) tc::tmem_ld16(tb + 64, r1);
-        if (jg < 2) tc::tmem_ld16(tb + 80 + jg * 16, r2);
-        if (jg < 3) tc::tmem_ld16(tb + 112 + jg * 16, r3);
-        tc::tmem_wait_ld();
-        float out[16];
-#pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          const int j = jg * 16 + jj;
+        for (int j = 0; j < 32; ++j) {
+          const int jg = j >> 4;
           float val = 0.f;
           if (jg < ar)
-            val = ar == 1 ? r1[jj] : (ar == 2 ? r2[jj] : r3[jj]);
+            val = ar == 1 ? r1[j & 15] : (ar == 2 ? r2[j] : r3[j]);
+          else if (jg == ar)
+            val = (is_q ? (j <= r) : (j < r)) ? dg[j] : 0.f;
+          out[j] = val;
+        }
+      } else {
+        float dg[32], r3[16];
+        tc::tmem_ld32(tb + 32, dg);
+        tc::tmem_ld16(tb + 144, r3);
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          const int j = 32 + jj, jg = j >> 4;
+          float val = 0.f;
+          if (jg < ar)
+            val = r3[jj & 15];  // only jg = 2 < ar = 3
           else if (jg == ar)
             val = (is_q ? (j <= r) : (j < r)) ? dg[jj] : 0.f;
           out[jj] = val;
         }
-        if (!is_q) {
+      }
+      const int jb = half * 32;
+      if (!is_q) {
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) nmat[r * 65 + jg * 16 + jj] = br * out[jj];
-        } else {
+        for (int q4 = 0; q4 < 8; ++q4)
+          *reinterpret_cast<float4*>(nmat + r * kLd + jb + q4 * 4) =
+              make_float4(br * out[q4 * 4], br * out[q4 * 4 + 1], br * out[q4 * 4 + 2],
+                          br * out[q4 * 4 + 3]);
+      } else {
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            *reinterpret_cast<float4*>(smem + OFF_MQK +
-                                       tc::sw128<4>(r, jg * 16 + q4 * 4, 64)) =
-                make_float4(out[q4 * 4], out[q4 * 4 + 1], out[q4 * 4 + 2], out[q4 * 4 + 3]);
-        }
+        for (int q4 = 0; q4 < 8; ++q4)
+          *reinterpret_cast<float4*>(smem + OFF_MQK + tc::sw128<4>(r, jb + q4 * 4, 64)) =
+              make_float4(out[q4 * 4], out[q4 * 4 + 1], out[q4 * 4 + 2], out[q4 * 4 + 3]);
       }
     }
     tc::fence_async_smem();
@@ -349,42 +481,7 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     {
       const float* N = reinterpret_cast<const float*>(smem + OFF_NMAT);
       float* X = reinterpret_cast<float*>(smem + OFF_XMAT);
-      float* Y = reinterpret_cast<float*>(smem + OFF_YBUF);
-      if (tid < 64) {
-        const int base = (tid >> 4) * 16, col = tid & 15;
-        float x[16];
-#pragma unroll
-        for (int rr = 0; rr < 16; ++rr) {
-          float acc = rr == col ? 1.f : 0.f;
-#pragma unroll
-          for (int jj = 0; jj < rr; ++jj) acc -= N[(base + rr) * 65 + base + jj] * x[jj];
-          x[rr] = acc;
-        }
-#pragma unroll
-        for (int rr = 0; rr < 16; ++rr) X[(base + rr) * 65 + base + col] = x[rr];
-      }
-      __syncthreads();
-      const int rr = tid >> 4, cc = tid & 15;
-      for (int a = 1; a < 4; ++a) {
-        for (int b = 0; b < a; ++b) {
-          float acc = 0.f;
-          for (int c = b; c < a; ++c) {
-#pragma unroll
-            for (int jj = 0; jj < 16; ++jj)
-              acc += N[(a * 16 + rr) * 65 + c * 16 + jj] * X[(c * 16 + jj) * 65 + b * 16 + cc];
-          }
-          Y[(b * 16 + rr) * 17 + cc] = acc;
-        }
-        __syncthreads();
-        for (int b = 0; b < a; ++b) {
-          float acc = 0.f;
-#pragma unroll
-          for (int kk = 0; kk < 16; ++kk)
-            acc += X[(a * 16 + rr) * 65 + a * 16 + kk] * Y[(b * 16 + kk) * 17 + cc];
-          X[(a * 16 + rr) * 65 + b * 16 + cc] = -acc;
-        }
-        __syncthreads();
-      }
+      invert_unit_lower64(N, X, reinterpret_cast<float*>(smem + OFF_ZBUF), tid);
       // T = X diag(beta) (lower triangle incl. diagonal) -> bf16 K-major [r][j]
       {
         const int r = tid >> 2, j0 = (tid & 3) * 16;
@@ -394,8 +491,8 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
 #pragma unroll
           for (int e = 0; e < 8; e += 2) {
             const int j = j0 + h8 * 8 + e;
-            const float x0 = j <= r ? X[r * 65 + j] * s_beta[j] : 0.f;
-            const float x1 = j + 1 <= r ? X[r * 65 + j + 1] * s_beta[j + 1] : 0.f;
+            const float x0 = j <= r ? X[r * kLd + j] * s_beta[j] : 0.f;
+            const float x1 = j + 1 <= r ? X[r * kLd + j + 1] * s_beta[j + 1] : 0.f;
             w[e >> 1] = pack_bf16x2(x0, x1);
           }
           *reinterpret_cast<uint4*>(smem + OFF_TM + tc::sw128<2>(r, j0 + h8 * 8, 64)) =
@@ -428,17 +525,16 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       const int c = warp * 32 + lane;
       const uint32_t tb = tmem + (static_cast<uint32_t>(warp * 32) << 16) + TM_W;
 #pragma unroll
-      for (int rg = 0; rg < 4; ++rg) {
-        float w[16];
-        tc::tmem_ld16(tb + rg * 16, w);
-        tc::tmem_wait_ld();
+      for (int rg = 0; rg < 2; ++rg) {
+        float w[32];
+        tc::tmem_ld32(tb + rg * 32, w);
 #pragma unroll
-        for (int h8 = 0; h8 < 2; ++h8) {
+        for (int h8 = 0; h8 < 4; ++h8) {
           uint32_t p[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e)
             p[e] = pack_bf16x2(-w[h8 * 8 + 2 * e], -w[h8 * 8 + 2 * e + 1]);
-          *reinterpret_cast<uint4*>(smem + OFF_NW + tc::sw128<2>(c, rg * 16 + h8 * 8, 128)) =
+          *reinterpret_cast<uint4*>(smem + OFF_NW + tc::sw128<2>(c, rg * 32 + h8 * 8, 128)) =
               make_uint4(p[0], p[1], p[2], p[3]);
         }
       }
@@ -446,13 +542,12 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     {
       const uint32_t tb = tmem + lane_off + TM_S + half * 64;
 #pragma unroll
-      for (int cg = 0; cg < 4; ++cg) {
-        float s[16];
-        tc::tmem_ld16(tb + cg * 16, s);
-        tc::tmem_wait_ld();
-        const int cb = half * 64 + cg * 16;
+      for (int cg = 0; cg < 2; ++cg) {
+        float s[32];
+        tc::tmem_ld32(tb + cg * 32, s);
+        const int cb = half * 64 + cg * 32;
 #pragma unroll
-        for (int h8 = 0; h8 < 2; ++h8) {
+        for (int h8 = 0; h8 < 4; ++h8) {
           uint32_t p[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) p[e] = pack_bf16x2(s[h8 * 8 + 2 * e], s[h8 * 8 + 2 * e + 1]);
@@ -460,8 +555,9 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
               make_uint4(p[0], p[1], p[2], p[3]);
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) s[i] *= s_gamma[cb + i];
-        tc::tmem_st16(tb + cg * 16, s);
+        for (int i = 0; i < 32; ++i) s[i] *= s_gamma[cb + i];
+        tc::tmem_st16(tb + cg * 32, s);
+        tc::tmem_st16(tb + cg * 32 + 16, s + 16);
       }
       tc::tmem_wait_st();
     }
@@ -508,19 +604,22 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     phase ^= 1;
     if (!ok) break;
 
-    // ---- P9: O to HBM (bf16) ---------------------------------------------
+    // ---- P9: O to HBM (bf16), staged through shared memory ----------------
     {
-      const uint32_t tb = tmem + lane_off + TM_O + half * 32;
+      // The Q*e^g tile is dead once P7 completed: reuse it for O as [r][m].
+      __nv_bfloat16* otile = reinterpret_cast<__nv_bfloat16*>(smem + OFF_QT);
+      float ov[32];
+      tc::tmem_ld32(tmem + lane_off + TM_O + half * 32, ov);
 #pragma unroll
-      for (int rg = 0; rg < 2; ++rg) {
-        float ov[16];
-        tc::tmem_ld16(tb + rg * 16, ov);
-        tc::tmem_wait_ld();
+      for (int i = 0; i < 32; ++i) otile[(half * 32 + i) * DV + m] = __float2bfloat16_rn(ov[i]);
+      __syncthreads();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int r = half * 32 + rg * 16 + i;
-          if (r < L) o[((size_t)(t0 + r) * H + head) * DV + m] = __float2bfloat16_rn(ov[i]);
-        }
+      for (int it = 0; it < 4; ++it) {
+        const int idx = it * kThreads + tid;
+        const int r = idx >> 4, c8 = idx & 15;
+        if (r < L)
+          *reinterpret_cast<uint4*>(o + ((size_t)(t0 + r) * H + head) * DV + c8 * 8) =
+              *reinterpret_cast<const uint4*>(otile + r * DV + c8 * 8);
       }
     }
     cta_sync_tc();
