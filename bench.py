@@ -142,52 +142,66 @@ def barrier(world):
     torch.cuda.synchronize()
 
 
-def cpu_oracle_prefill(budget_s=12.0, seed=0):
-    """Time the fp64 oracle on a bounded sample of the prefill workload: all
-    B*H chains over their first `n_tok` tokens, n_tok sized to about
-    `budget_s` seconds from a short calibration run."""
+def _oracle_sample(n_tok, seed=0):
     import torch
-    import oracle
     from gated_delta_rule_61_b200.inputs import prefill_inputs
     P = PREFILL
-    cores = oracle.default_threads()
+    return prefill_inputs(P["B"], n_tok, P["H"], P["dk"], P["dv"], dtype=torch.bfloat16,
+                          seed=seed, init_std=P["init_std"])
 
-    def run(n_tok):
-        inp = prefill_inputs(P["B"], n_tok, P["H"], P["dk"], P["dv"], dtype=torch.bfloat16,
-                             seed=seed, init_std=P["init_std"])
-        t0 = time.perf_counter()
-        oracle.kda_forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
-                           init_state=inp["init_state"], n_threads=cores)
-        return time.perf_counter() - t0
 
+def _oracle_run(inp, cores):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.kda_forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                       init_state=inp["init_state"], n_threads=cores)
+    return time.perf_counter() - t0
+
+
+def _oracle_tokens_for(budget_s, cores):
+    """Tokens per chain (all B*H chains) the oracle covers in about budget_s."""
     cal = 32
-    dt = run(cal)
-    n_tok = int(max(cal, min(P["T"], cal * budget_s / max(dt, 1e-6))))
-    dt = run(n_tok)
-    tok_s = P["B"] * n_tok / dt
-    return tok_s, cores, n_tok, dt
+    dt = _oracle_run(_oracle_sample(cal), cores)
+    return int(max(cal, min(PREFILL["T"], cal * budget_s / max(dt, 1e-6))))
+
+
+def cpu_oracle_prefill(budget_s=12.0, seed=0):
+    """Time the fp64 oracle on a bounded sample of the prefill workload: all
+    B*H chains over their first n_tok tokens, n_tok sized to about budget_s
+    seconds from a short calibration run."""
+    import oracle
+    cores = oracle.default_threads()
+    n_tok = _oracle_tokens_for(budget_s, cores)
+    dt = _oracle_run(_oracle_sample(n_tok, seed), cores)
+    return PREFILL["B"] * n_tok / dt, cores, n_tok, dt
 
 
 def bench_reference(args):
-    world, rank, _ = (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
-                      0)
+    """The fp64 oracle as the reference arm: rank 0 only, each step a bounded
+    sample of the workload sized so the whole run takes about two minutes."""
+    import oracle
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    times, n_toks, cores = [], [], None
-    for i in range(args.warmup + args.steps):
-        tok_s, cores, n_tok, dt = cpu_oracle_prefill(budget_s=args.ref_budget, seed=i)
-        if i >= args.warmup:
-            times.append(tok_s)
-            n_toks.append(n_tok)
-    value = statistics.median(times)
+    cores = oracle.default_threads()
+    per_step = max(0.05, min(args.ref_budget, 120.0 / (args.steps + args.warmup)))
+    n_tok = _oracle_tokens_for(per_step, cores)
+    inp = _oracle_sample(n_tok)
+    for _ in range(args.warmup):
+        _oracle_run(inp, cores)
+    times = [_oracle_run(inp, cores) for _ in range(args.steps)]
+    total = sum(times)
     P = PREFILL
-    sample = ("all %d (batch, head) chains, first %d of %d tokens, fp64 oracle"
-              % (P["B"] * P["H"], min(n_toks), P["T"]))
+    value = P["B"] * n_tok * args.steps / total
+    sample = ("all %d (batch, head) chains, first %d of %d tokens per step, fp64 oracle"
+              % (P["B"] * P["H"], n_tok, P["T"]))
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * P["B"] * P["T"] / value, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "KDA prefill B=4 T=8192 H=16 dk=dv=128 bf16 inputs, C=64",
+            "config": {"workload": "KDA prefill B=4 T=8192 H=16 dk=dv=128 bf16 q/k/v, fp32 "
+                                   "gates and state, chunk C=64 (per GPU)",
                        "global_batch": P["B"], "seq_len": P["T"], "heads": P["H"],
                        "parallelism": "replicas"},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,

@@ -5,14 +5,14 @@
 // or Parallelizing Linear Transformers with Delta Rule" (cut the sequence into
 // chunks of C tokens; inside a chunk the deltas come from a unit lower-
 // triangular system built from the keys (the UT/WY form of the Householder
-// products), across chunks the state carries everything: "C = 64 or 128 ...
-// tensor-core instructions such as UMMA"), with the per-channel decay of
-// "Gated Delta Net" (cumulative decay is a multiplicative prefix sum) and
-// "KDA / Kimi Linear"; the ai-flip.ru KDA explainer (channel-wise diagonal
-// gate; chunked computation on tensor cores). Derived for the KDA step
-// S_t = (I - b k k^T) Diag(a_t) S_{t-1} + b k v^T, with g the within-chunk
-// cumulative sum of log_alpha per key channel and S0 the state entering the
-// chunk:
+// products), across chunks the state carries everything; C is 64 or 128 to
+// match tensor-core instruction granularity, UMMA being one example), with the
+// per-channel decay of "Gated Delta Net" (cumulative decay is a multiplicative
+// prefix sum) and "KDA / Kimi Linear"; the ai-flip.ru KDA explainer
+// (channel-wise diagonal gate; chunked computation on tensor cores). Derived
+// for the KDA step S_t = (I - b k k^T) Diag(a_t) S_{t-1} + b k v^T, with g the
+// within-chunk cumulative sum of log_alpha per key channel and S0 the state
+// entering the chunk:
 //   M_kk[r,j] = sum_c k_rc k_jc e^{g_rc - g_jc} (j < r)
 //   M_qk[r,j] = sum_c q_rc k_jc e^{g_rc - g_jc} (j <= r)
 //   X = (I + diag(beta) M_kk)^-1,  T = X diag(beta)
@@ -31,22 +31,25 @@
 // sub-chunk a). Entries outside the blocks each row needs are ignored.
 //
 // Precision. Gram, T, W, U and the products with the state S0 use bf16
-// operands with fp32 accumulation; the state update (K^T D) and the
+// operands with fp32 accumulation; the state update (K~^T D) and the
 // output's correction (M_qk D) read D straight from tensor memory as tf32,
 // and the state itself stays fp32 in tensor memory for the whole sequence.
 //
-// Layout. One CTA (256 threads) per (sequence, head) chain, walking its
-// chunks in order. Tensor memory (512 columns, lanes = dv index m for the
-// state-sized accumulators):
+// Layout. One CTA (512 threads = 16 warps) per (sequence, head) chain,
+// walking its chunks in order. Warp w reaches tensor-memory lanes
+// [32 (w % 4), +32); the four warps sharing a lane quadrant split the columns.
+// Tensor memory (512 columns, lanes = dv index m for the state-sized
+// accumulators):
 //   [0,128)   S^T (fp32 state, lane m, column c)
 //   [128,192) U^T, then D^T = U^T - (W S0)^T   (lane m, column = position)
 //   [192,256) O^T                              (lane m, column = position)
 //   [256,416) Gram result (lanes 0..63 k rows, 64..127 q rows); later W^T
-// Per chunk: (P1) gates and operand tiles from global memory; (P2) Gram MMA;
-// (P3) rows of M_kk and M_qk out of tensor memory; (P4) block forward
-// substitution for X on CUDA cores; (P5) W^T and U^T MMAs; (P6) -W to shared
-// memory, S0 to bf16 and the decay of the fp32 state; (P7) D and the first
-// part of O; (P8) tf32 state update and output correction; (P9) O to HBM.
+// Per chunk n: (P1) gates and operand tiles; (P2) Gram MMA, during which the
+// previous chunk's output leaves tensor memory for HBM; (P3) rows of M_kk and
+// M_qk; (P4) block inverse for X on CUDA cores; (P5) W^T and U^T MMAs, during
+// which the state is copied to bf16 and decayed in place; -W to shared
+// memory; (P7) D and the first part of O; (P8) tf32 state update and output
+// correction.
 #include "kda_common.cuh"
 #include "kda_tc.cuh"
 
@@ -54,29 +57,29 @@ namespace kda {
 namespace chunk64 {
 
 constexpr int C = 64, DK = 128, DV = 128;
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr float kLogAlphaMin = -10.0f;
 constexpr uint64_t kMaxWaitNs = 1000000000ull;  // 1 s per bounded wait
 
 // Shared memory (byte offsets from a 1024-aligned base).
-constexpr uint32_t OFF_SB = 0;         // S0 bf16, K-major [m][c]            32768
-constexpr uint32_t OFF_QT = 32768;     // Q*e^g bf16, K-major [r][c]          16384
-constexpr uint32_t OFF_KT = 49152;     // K*e^(glast-g) fp32, K-major [c][j]  32768
-constexpr uint32_t OFF_BK = 81920;     // K*e^g bf16, MN-major [j][c]         16384
-constexpr uint32_t OFF_VV = 98304;     // V bf16, MN-major [j][m]             16384
-constexpr uint32_t OFF_AG = 114688;    // Gram A bf16 K-major [128][c]        32768
+constexpr uint32_t OFF_SB = 0;         // S0 bf16, K-major [m][c] (also O staging)  32768
+constexpr uint32_t OFF_QT = 32768;     // Q*e^g bf16, K-major [r][c]                 16384
+constexpr uint32_t OFF_KT = 49152;     // K*e^(glast-g) fp32, K-major [c][j]         32768
+constexpr uint32_t OFF_BK = 81920;     // K*e^g bf16, MN-major [j][c]                16384
+constexpr uint32_t OFF_VV = 98304;     // V bf16, MN-major [j][m]                    16384
+constexpr uint32_t OFF_AG = 114688;    // Gram A bf16 K-major [128][c]               32768
 constexpr uint32_t OFF_MQK = OFF_AG;           // after the Gram MMA: M_qk fp32 K-major [r][j]
 constexpr uint32_t OFF_TM = OFF_AG + 16384;    // T bf16 K-major [r][j]
-constexpr uint32_t OFF_BG = 147456;    // Gram B bf16 K-major [160][c]        40960
+constexpr uint32_t OFF_BG = 147456;    // Gram B bf16 K-major [160][c]               40960
 constexpr int kLd = 68;                        // row stride (floats) of the solve's matrices
-constexpr uint32_t OFF_NMAT = OFF_BG;          // after the Gram MMA: diag(beta) M_kk, fp32 [64][68]
+constexpr uint32_t OFF_NMAT = OFF_BG;          // after the Gram MMA: diag(beta) M_kk [64][68]
 constexpr uint32_t OFF_XMAT = OFF_BG + 17408;  // X, fp32 [64][68]
 constexpr uint32_t OFF_ZBUF = OFF_BG + 34816;  // block products, fp32 [32][34]
 constexpr uint32_t OFF_NW = OFF_BG;            // after the solve: -W^T bf16 MN-major [c][r]
 constexpr uint32_t OFF_MISC = 188416;
-constexpr uint32_t MISC_GAMMA = 0, MISC_BETA = 512, MISC_TOT = 768, MISC_MID = 2816,
-                   MISC_GLAST = 4864, MISC_MBAR = 5376, MISC_TMEM = 5384;
-constexpr uint32_t kSmemBytes = OFF_MISC + 5392 + 1024;
+constexpr uint32_t MISC_GAMMA = 0, MISC_BETA = 512, MISC_TOT = 768, MISC_GF = 4864,
+                   MISC_GL = 8960, MISC_MBAR = 13056, MISC_TMEM = 13064;
+constexpr uint32_t kSmemBytes = OFF_MISC + 13072 + 1024;
 
 // Tensor-memory columns.
 constexpr uint32_t TM_S = 0, TM_D = 128, TM_O = 192, TM_G = 256, TM_W = 256;
@@ -86,8 +89,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&p);
 }
 
-// All threads wait for the MMA barrier phase; thread 0 spins (bounded) and
-// the result is shared through the CTA barrier.
+// Thread 0 spins (bounded) on the MMA barrier phase; the outcome is shared
+// through the CTA barrier.
 __device__ __forceinline__ bool cta_wait(uint32_t mbar, uint32_t parity, int code) {
   int fail = 0;
   if (threadIdx.x == 0) fail = !tc::mbar_wait_bounded(mbar, parity, kMaxWaitNs) ? 1 : 0;
@@ -108,7 +111,7 @@ __device__ __forceinline__ void cta_sync_tc() {
 // [[A, 0], [C, D]] the inverse is [[A^-1, 0], [-D^-1 C A^-1, D^-1]].
 // Level 1 inverts the four 16 x 16 diagonal blocks by forward substitution,
 // level 2 fills the two 16 x 16 blocks below them, level 3 the 32 x 32 block.
-// All 256 threads take part; entries above the diagonal are never read.
+// Entries above the diagonal are never read.
 __device__ __forceinline__ void invert_diag_block(const float* N, float* X, int t) {
   const int base = (t >> 4) * 16, col = t & 15;
   float x[16];
@@ -133,58 +136,76 @@ __device__ __forceinline__ void invert_unit_lower64(const float* N, float* X, fl
   __syncthreads();
   // Level 2: blocks (1,0) and (3,2): Z_p = N_{b a} X_{a a}, X_{b a} = -X_{b b} Z_p.
   {
-    const int p = t >> 7, rr = (t >> 3) & 15, cc = (t & 7) * 2;
+    const int p = t >> 8, rr = (t >> 4) & 15, cc = t & 15;
     const int a = 2 * p * 16, b = a + 16;
     float z0 = 0.f, z1 = 0.f;
 #pragma unroll
-    for (int kk = 0; kk < 16; ++kk) {
-      const float nv = N[(b + rr) * kLd + a + kk];
-      const float2 xv = *reinterpret_cast<const float2*>(X + (a + kk) * kLd + a + cc);
-      z0 += nv * xv.x;
-      z1 += nv * xv.y;
+    for (int kk = 0; kk < 16; kk += 2) {
+      z0 += N[(b + rr) * kLd + a + kk] * X[(a + kk) * kLd + a + cc];
+      z1 += N[(b + rr) * kLd + a + kk + 1] * X[(a + kk + 1) * kLd + a + cc];
     }
-    *reinterpret_cast<float2*>(Z + (p * 16 + rr) * 34 + cc) = make_float2(z0, z1);
+    Z[(p * 16 + rr) * 34 + cc] = z0 + z1;
     __syncthreads();
     float x0 = 0.f, x1 = 0.f;
 #pragma unroll
-    for (int kk = 0; kk < 16; ++kk) {
-      const float xv = X[(b + rr) * kLd + b + kk];
-      const float2 zv = *reinterpret_cast<const float2*>(Z + (p * 16 + kk) * 34 + cc);
-      x0 += xv * zv.x;
-      x1 += xv * zv.y;
+    for (int kk = 0; kk < 16; kk += 2) {
+      x0 += X[(b + rr) * kLd + b + kk] * Z[(p * 16 + kk) * 34 + cc];
+      x1 += X[(b + rr) * kLd + b + kk + 1] * Z[(p * 16 + kk + 1) * 34 + cc];
     }
-    *reinterpret_cast<float2*>(X + (b + rr) * kLd + a + cc) = make_float2(-x0, -x1);
+    X[(b + rr) * kLd + a + cc] = -(x0 + x1);
     __syncthreads();
   }
   // Level 3: Z = N[32:64, 0:32] X[0:32, 0:32];  X[32:64, 0:32] = -X[32:64, 32:64] Z.
   {
-    const int r2 = (t >> 4) * 2, c2 = (t & 15) * 2;
-    float z00 = 0.f, z01 = 0.f, z10 = 0.f, z11 = 0.f;
+    const int r = t >> 4, c2 = (t & 15) * 2;
+    float z0 = 0.f, z1 = 0.f, y0 = 0.f, y1 = 0.f;
 #pragma unroll
-    for (int kk = 0; kk < 32; ++kk) {
-      const float n0 = N[(32 + r2) * kLd + kk], n1 = N[(33 + r2) * kLd + kk];
-      const float2 xv = *reinterpret_cast<const float2*>(X + kk * kLd + c2);
-      const bool live = kk >= c2;  // X[0:32,0:32] is lower triangular
-      const float x0 = live ? xv.x : 0.f, x1 = kk >= c2 + 1 ? xv.y : 0.f;
-      z00 += n0 * x0; z01 += n0 * x1;
-      z10 += n1 * x0; z11 += n1 * x1;
+    for (int kk = 0; kk < 32; kk += 2) {
+      const float n0 = N[(32 + r) * kLd + kk], n1 = N[(32 + r) * kLd + kk + 1];
+      const float2 xa = *reinterpret_cast<const float2*>(X + kk * kLd + c2);
+      const float2 xb = *reinterpret_cast<const float2*>(X + (kk + 1) * kLd + c2);
+      // X[0:32, 0:32] is lower triangular: entry (kk, c) is live for kk >= c.
+      z0 += n0 * (kk >= c2 ? xa.x : 0.f);
+      z1 += n0 * (kk >= c2 + 1 ? xa.y : 0.f);
+      y0 += n1 * (kk + 1 >= c2 ? xb.x : 0.f);
+      y1 += n1 * (kk + 1 >= c2 + 1 ? xb.y : 0.f);
     }
-    *reinterpret_cast<float2*>(Z + r2 * 34 + c2) = make_float2(z00, z01);
-    *reinterpret_cast<float2*>(Z + (r2 + 1) * 34 + c2) = make_float2(z10, z11);
+    *reinterpret_cast<float2*>(Z + r * 34 + c2) = make_float2(z0 + y0, z1 + y1);
     __syncthreads();
-    float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
+    float x0 = 0.f, x1 = 0.f, w0 = 0.f, w1 = 0.f;
 #pragma unroll
-    for (int kk = 0; kk < 32; ++kk) {
-      const bool l0 = kk <= r2, l1 = kk <= r2 + 1;  // X[32:64,32:64] is lower triangular
-      const float d0 = l0 ? X[(32 + r2) * kLd + 32 + kk] : 0.f;
-      const float d1 = l1 ? X[(33 + r2) * kLd + 32 + kk] : 0.f;
-      const float2 zv = *reinterpret_cast<const float2*>(Z + kk * 34 + c2);
-      x00 += d0 * zv.x; x01 += d0 * zv.y;
-      x10 += d1 * zv.x; x11 += d1 * zv.y;
+    for (int kk = 0; kk < 32; kk += 2) {
+      // X[32:64, 32:64] is lower triangular: (r, kk) is live for kk <= r.
+      const float d0 = kk <= r ? X[(32 + r) * kLd + 32 + kk] : 0.f;
+      const float d1 = kk + 1 <= r ? X[(32 + r) * kLd + 33 + kk] : 0.f;
+      const float2 za = *reinterpret_cast<const float2*>(Z + kk * 34 + c2);
+      const float2 zb = *reinterpret_cast<const float2*>(Z + (kk + 1) * 34 + c2);
+      x0 += d0 * za.x; x1 += d0 * za.y;
+      w0 += d1 * zb.x; w1 += d1 * zb.y;
     }
-    *reinterpret_cast<float2*>(X + (32 + r2) * kLd + c2) = make_float2(-x00, -x01);
-    *reinterpret_cast<float2*>(X + (33 + r2) * kLd + c2) = make_float2(-x10, -x11);
+    *reinterpret_cast<float2*>(X + (32 + r) * kLd + c2) = make_float2(-(x0 + w0), -(x1 + w1));
     __syncthreads();
+  }
+}
+
+// O^T (lane m, column r) of one chunk -> bf16 [r][m] in shared memory ->
+// coalesced 16-byte stores of the first L rows.
+__device__ __forceinline__ void store_output(uint32_t tmem, uint32_t lane_off, int grp, int m,
+                                             uint8_t* stage, __nv_bfloat16* o, long long t0,
+                                             int L, int H, int head) {
+  __nv_bfloat16* otile = reinterpret_cast<__nv_bfloat16*>(stage);
+  float ov[16];
+  tc::tmem_ld16(tmem + lane_off + TM_O + grp * 16, ov);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) otile[(grp * 16 + i) * DV + m] = __float2bfloat16_rn(ov[i]);
+  __syncthreads();
+#pragma unroll
+  for (int it = 0; it < 2; ++it) {
+    const int idx = it * kThreads + threadIdx.x;
+    const int r = idx >> 4, c8 = idx & 15;
+    if (r < L)
+      *reinterpret_cast<uint4*>(o + ((size_t)(t0 + r) * H + head) * DV + c8 * 8) =
+          *reinterpret_cast<const uint4*>(otile + r * DV + c8 * 8);
   }
 }
 
@@ -200,9 +221,9 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
   const uint32_t sbase = tc::smem_u32(smem);
   float* s_gamma = reinterpret_cast<float*>(smem + OFF_MISC + MISC_GAMMA);
   float* s_beta = reinterpret_cast<float*>(smem + OFF_MISC + MISC_BETA);
-  float* s_tot = reinterpret_cast<float*>(smem + OFF_MISC + MISC_TOT);
-  float* s_mid = reinterpret_cast<float*>(smem + OFF_MISC + MISC_MID);
-  float* s_glast = reinterpret_cast<float*>(smem + OFF_MISC + MISC_GLAST);
+  float* s_tot = reinterpret_cast<float*>(smem + OFF_MISC + MISC_TOT);   // [8][128]
+  float* s_gf = reinterpret_cast<float*>(smem + OFF_MISC + MISC_GF);     // [8][128]
+  float* s_gl = reinterpret_cast<float*>(smem + OFF_MISC + MISC_GL);     // [8][128]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC + MISC_TMEM);
   const uint32_t mbar = sbase + OFF_MISC + MISC_MBAR;
 
@@ -226,50 +247,43 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
   uint32_t phase = 0;
   bool ok = true;
 
-  // TMEM access: warp w reaches lanes [32 (w % 4), +32); the two warps that
-  // share a lane quadrant split the columns of 128-column passes.
-  const int quad = warp & 3, half = warp >> 2;
+  const int quad = warp & 3, grp = warp >> 2;
   const int m = quad * 32 + lane;
   const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
   const size_t state_off = ((size_t)seq * H + head) * DK * DV;
 
-  // Initial state: S^T[m][c] = S0[c][m].
+  // Initial state: S^T[m][c] = S0[c][m]; this warp covers columns [32 grp, +32).
   {
-    const uint32_t tb = tmem + lane_off + TM_S + half * 64;
+    float vals[32];
 #pragma unroll
-    for (int cg = 0; cg < 4; ++cg) {
-      float vals[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int c = half * 64 + cg * 16 + i;
-        vals[i] = init_state ? init_state[state_off + (size_t)c * DV + m] : 0.f;
-      }
-      tc::tmem_st16(tb + cg * 16, vals);
+    for (int i = 0; i < 32; ++i) {
+      const int c = grp * 32 + i;
+      vals[i] = init_state ? init_state[state_off + (size_t)c * DV + m] : 0.f;
     }
+    tc::tmem_st16(tmem + lane_off + TM_S + grp * 32, vals);
+    tc::tmem_st16(tmem + lane_off + TM_S + grp * 32 + 16, vals + 16);
     tc::tmem_wait_st();
   }
   cta_sync_tc();
 
   const long long len = t_end - t_begin;
   const int n_chunks = (int)((len + C - 1) / C);
-  const int pr = tid & 63, sub = tid >> 6, c0 = 2 * pr;  // P1 mapping
+  // P1 mapping: channel pair (c0, c0 + 1), rows [8 rg, 8 rg + 8) of sub-chunk rg / 2.
+  const int pr = tid & 63, rg = tid >> 6, sub = rg >> 1, c0 = 2 * pr;
 
   for (int n = 0; n < n_chunks; ++n) {
     const long long t0 = t_begin + (long long)n * C;
     const int L = (int)((t_end - t0) < C ? (t_end - t0) : C);
 
     // ---- P1: cumulative gates and operand tiles --------------------------
-    // Every global load of this thread's 16 rows is issued before any use,
-    // so the rows' latencies overlap (the chunk was prefetched into L2 while
-    // the previous chunk ran).
-    float g0[16], g1[16];
-    uint32_t kr[16], qr[16], vr[16];
-    float bt[16];
+    float g0[8], g1[8];
+    uint32_t kr[8], qr[8], vr[8];
+    float bt[8];
     {
-      float2 lr[16];
+      float2 lr[8];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int r = sub * 16 + i;
+      for (int i = 0; i < 8; ++i) {
+        const int r = rg * 8 + i;
         lr[i] = make_float2(0.f, 0.f);
         kr[i] = qr[i] = vr[i] = 0u;
         bt[i] = 0.f;
@@ -284,54 +298,65 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       }
       float run0 = 0.f, run1 = 0.f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < 8; ++i) {
         run0 += fmaxf(lr[i].x, kLogAlphaMin);
         run1 += fmaxf(lr[i].y, kLogAlphaMin);
         g0[i] = run0;
         g1[i] = run1;
       }
-      s_tot[sub * 128 + c0] = run0;
-      s_tot[sub * 128 + c0 + 1] = run1;
+      s_tot[rg * 128 + c0] = run0;
+      s_tot[rg * 128 + c0 + 1] = run1;
     }
     __syncthreads();
-    float m0, m1;
     {
       float off0 = 0.f, off1 = 0.f;
-      for (int b = 0; b < sub; ++b) {
+      for (int b = 0; b < rg; ++b) {
         off0 += s_tot[b * 128 + c0];
         off1 += s_tot[b * 128 + c0 + 1];
       }
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < 8; ++i) {
         g0[i] += off0;
         g1[i] += off1;
       }
-      m0 = 0.5f * (g0[0] + g0[15]);
-      m1 = 0.5f * (g1[0] + g1[15]);
-      s_mid[sub * 128 + c0] = m0;
-      s_mid[sub * 128 + c0 + 1] = m1;
-      if (sub == 3) {
-        s_glast[c0] = g0[15];
-        s_glast[c0 + 1] = g1[15];
-        s_gamma[c0] = expf(g0[15]);
-        s_gamma[c0 + 1] = expf(g1[15]);
+      s_gf[rg * 128 + c0] = g0[0];
+      s_gf[rg * 128 + c0 + 1] = g1[0];
+      s_gl[rg * 128 + c0] = g0[7];
+      s_gl[rg * 128 + c0 + 1] = g1[7];
+      if (rg == 7) {
+        s_gamma[c0] = __expf(g0[7]);
+        s_gamma[c0 + 1] = __expf(g1[7]);
+      }
+      if (pr == 0) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s_beta[rg * 8 + i] = bt[i];
       }
     }
     __syncthreads();
     {
-      const float em0 = expf(m0), em1 = expf(m1);
-      const float kt0 = expf(s_glast[c0] - m0), kt1 = expf(s_glast[c0 + 1] - m1);
+      // Sub-chunk midpoints m_a = (g at its first row + g at its last row) / 2.
+      float mid0[4], mid1[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        mid0[a] = 0.5f * (s_gf[(2 * a) * 128 + c0] + s_gl[(2 * a + 1) * 128 + c0]);
+        mid1[a] = 0.5f * (s_gf[(2 * a) * 128 + c0 + 1] + s_gl[(2 * a + 1) * 128 + c0 + 1]);
+      }
+      const float m0 = sub == 0 ? mid0[0] : sub == 1 ? mid0[1] : sub == 2 ? mid0[2] : mid0[3];
+      const float m1 = sub == 0 ? mid1[0] : sub == 1 ? mid1[1] : sub == 2 ? mid1[2] : mid1[3];
+      const float glast0 = s_gl[7 * 128 + c0], glast1 = s_gl[7 * 128 + c0 + 1];
+      const float em0 = __expf(m0), em1 = __expf(m1);
+      const float kt0 = __expf(glast0 - m0), kt1 = __expf(glast1 - m1);
       float rho0[4], rho1[4];
 #pragma unroll
       for (int ap = 0; ap < 4; ++ap) {
-        rho0[ap] = ap > sub ? expf(s_mid[ap * 128 + c0] - m0) : 0.f;
-        rho1[ap] = ap > sub ? expf(s_mid[ap * 128 + c0 + 1] - m1) : 0.f;
+        rho0[ap] = ap > sub ? __expf(mid0[ap] - m0) : 0.f;
+        rho1[ap] = ap > sub ? __expf(mid1[ap] - m1) : 0.f;
       }
-      float kt_c0[16], kt_c1[16];
-      // Swizzled byte offsets of this thread's rows (r = 16 sub + i): (r & 7) = (i & 7)
-      // and (r >> 3) = 2 sub + (i >> 3), so only (chunk ^ (i & 7)) varies at run time.
+      float kt_c0[8], kt_c1[8];
+      // Swizzled byte offsets of this thread's rows r = 8 rg + i: (r & 7) = i and
+      // (r >> 3) = rg, so only (chunk ^ i) varies at run time.
       const int xr = (c0 & 63) >> 3;
-      const uint32_t colb = (uint32_t)((c0 & 7) * 2) + (uint32_t)sub * 2048u;
+      const uint32_t colb = (uint32_t)((c0 & 7) * 2) + (uint32_t)rg * 1024u;
       const uint32_t sl = (uint32_t)(c0 >> 6);
       uint8_t* const pAGk = smem + OFF_AG + sl * 16384u + colb;
       uint8_t* const pBGe = smem + OFF_BG + sl * 20480u + colb;
@@ -339,14 +364,11 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       uint8_t* const pBK = smem + OFF_BK + sl * 8192u + colb;
       uint8_t* const pVV = smem + OFF_VV + sl * 8192u + colb;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int r = sub * 16 + i;
-        const uint32_t ro = (uint32_t)((i >> 3) * 1024 + (i & 7) * 128) +
-                            ((uint32_t)(xr ^ (i & 7)) << 4);
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t ro = (uint32_t)(i * 128) + ((uint32_t)(xr ^ i) << 4);
         // bf16 pairs widen exactly: low half << 16, high half masked.
         const float k0 = __uint_as_float(kr[i] << 16), k1 = __uint_as_float(kr[i] & 0xffff0000u);
         const float q0 = __uint_as_float(qr[i] << 16), q1 = __uint_as_float(qr[i] & 0xffff0000u);
-        if (pr == 0) s_beta[r] = bt[i];
         const float f0 = __expf(g0[i] - m0), f1 = __expf(g1[i] - m1);
         const float fi0 = __expf(m0 - g0[i]), fi1 = __expf(m1 - g1[i]);
         *reinterpret_cast<uint32_t*>(pAGk + ro) = pack_bf16x2(k0 * f0, k1 * f1);
@@ -368,10 +390,10 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         kt_c0[i] = e0 * kt0;
         kt_c1[i] = e1 * kt1;
       }
-      // K~ as a K-major tf32 operand [c][j]: 16 consecutive positions per channel.
+      // K~ as a K-major tf32 operand [c][j]: 8 consecutive positions per channel.
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        const int j = sub * 16 + q4 * 4;
+      for (int q4 = 0; q4 < 2; ++q4) {
+        const int j = rg * 8 + q4 * 4;
         *reinterpret_cast<float4*>(smem + OFF_KT + tc::sw128<4>(c0, j, 128)) =
             make_float4(kt_c0[q4 * 4], kt_c0[q4 * 4 + 1], kt_c0[q4 * 4 + 2], kt_c0[q4 * 4 + 3]);
         *reinterpret_cast<float4*>(smem + OFF_KT + tc::sw128<4>(c0 + 1, j, 128)) =
@@ -381,7 +403,8 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     tc::fence_async_smem();
     cta_sync_tc();
 
-    // ---- P2: Gram MMA (M=128, N=160, K=128) ------------------------------
+    // ---- P2: Gram MMA (M=128, N=160, K=128); meanwhile the previous chunk's
+    // output goes to HBM (staged in the S0 bf16 tile, dead until P5) --------
     if (tid == 0) {
       constexpr uint32_t idesc = tc::make_idesc(1, 0, 0, 128, 160);
 #pragma unroll
@@ -394,24 +417,20 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       }
       tc::mma_commit(mbar);
     }
+    if (n > 0) store_output(tmem, lane_off, grp, m, smem + OFF_SB, o, t0 - C, C, H, head);
     if (n + 1 < n_chunks) {  // warm L2 with the next chunk's rows
       const long long t1 = t0 + C;
-      const int row = tid >> 2, part = tid & 3;
+      const int row = tid >> 3, part = tid & 7;
       if (t1 + row < t_end) {
         const size_t tok = (size_t)(t1 + row) * H + head;
-        if (part == 0) {
-          tc::prefetch_l2(q + tok * DK);
-          tc::prefetch_l2(q + tok * DK + 64);
-        } else if (part == 1) {
-          tc::prefetch_l2(k + tok * DK);
-          tc::prefetch_l2(k + tok * DK + 64);
-        } else if (part == 2) {
-          tc::prefetch_l2(v + tok * DV);
-          tc::prefetch_l2(v + tok * DV + 64);
+        if (part < 2) tc::prefetch_l2(q + tok * DK + 64 * part);
+        else if (part < 4) tc::prefetch_l2(k + tok * DK + 64 * (part - 2));
+        else if (part < 6) tc::prefetch_l2(v + tok * DV + 64 * (part - 4));
+        else tc::prefetch_l2(log_alpha + tok * DK + 64 * (part - 6));
+        if (part == 6) tc::prefetch_l2(log_alpha + tok * DK + 32);
+        if (part == 7) {
+          tc::prefetch_l2(log_alpha + tok * DK + 96);
           tc::prefetch_l2(beta + tok);
-        } else {
-#pragma unroll
-          for (int l = 0; l < 4; ++l) tc::prefetch_l2(log_alpha + tok * DK + 32 * l);
         }
       }
     }
@@ -420,90 +439,69 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     if (!ok) break;
 
     // ---- P3: rows of M_kk (lanes 0..63) and M_qk (lanes 64..127) ---------
-    // Warp pair (quad, half): half 0 assembles columns j < 32, half 1 j >= 32.
+    // Warp (quad, grp) assembles columns j in [16 grp, 16 grp + 16).
     {
-      const int row = quad * 32 + lane;
+      const int row = m;
       const bool is_q = row >= 64;
       const int r = row & 63, ar = r >> 4;
+      const int jg = grp;
       const uint32_t tb = tmem + lane_off + TM_G;
-      const float br = s_beta[r];
-      float* nmat = reinterpret_cast<float*>(smem + OFF_NMAT);
-      float out[32];
-      if (half == 0) {
-        float dg[32], r1[16], r2[32], r3[32];
-        tc::tmem_ld32(tb + 0, dg);
-        tc::tmem_ld16(tb + 64, r1);
-        tc::tmem_ld32(tb + 80, r2);
-        tc::tmem_ld32(tb + 112, r3);
+      // diag block columns, then the R sets that cover columns of group jg.
+      const uint32_t c_r1 = 64 + 16 * jg, c_r2 = 80 + 16 * jg, c_r3 = 112 + 16 * jg;
+      float vv[64];
+      tc::tmem_ld16x4(tb + 16 * jg, tb + (jg == 0 ? c_r1 : 16 * jg),
+                      tb + (jg <= 1 ? c_r2 : 16 * jg), tb + (jg <= 2 ? c_r3 : 16 * jg), vv);
+      float out[16];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int jg = j >> 4;
-          float val = 0.f;
-          if (jg < ar)
-            val = ar == 1 ? r1[j & 15] : (ar == 2 ? r2[j] : r3[j]);
-          else if (jg == ar)
-            val = (is_q ? (j <= r) : (j < r)) ? dg[j] : 0.f;
-          out[j] = val;
-        }
-      } else {
-        float dg[32], r3[16];
-        tc::tmem_ld32(tb + 32, dg);
-        tc::tmem_ld16(tb + 144, r3);
-#pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const int j = 32 + jj, jg = j >> 4;
-          float val = 0.f;
-          if (jg < ar)
-            val = r3[jj & 15];  // only jg = 2 < ar = 3
-          else if (jg == ar)
-            val = (is_q ? (j <= r) : (j < r)) ? dg[jj] : 0.f;
-          out[jj] = val;
-        }
+      for (int jj = 0; jj < 16; ++jj) {
+        const int j = jg * 16 + jj;
+        float val = 0.f;
+        if (jg < ar)
+          val = ar == 1 ? vv[16 + jj] : (ar == 2 ? vv[32 + jj] : vv[48 + jj]);
+        else if (jg == ar)
+          val = (is_q ? (j <= r) : (j < r)) ? vv[jj] : 0.f;
+        out[jj] = val;
       }
-      const int jb = half * 32;
       if (!is_q) {
+        const float br = s_beta[r];
+        float* nmat = reinterpret_cast<float*>(smem + OFF_NMAT);
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4)
-          *reinterpret_cast<float4*>(nmat + r * kLd + jb + q4 * 4) =
+        for (int q4 = 0; q4 < 4; ++q4)
+          *reinterpret_cast<float4*>(nmat + r * kLd + jg * 16 + q4 * 4) =
               make_float4(br * out[q4 * 4], br * out[q4 * 4 + 1], br * out[q4 * 4 + 2],
                           br * out[q4 * 4 + 3]);
       } else {
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4)
-          *reinterpret_cast<float4*>(smem + OFF_MQK + tc::sw128<4>(r, jb + q4 * 4, 64)) =
+        for (int q4 = 0; q4 < 4; ++q4)
+          *reinterpret_cast<float4*>(smem + OFF_MQK + tc::sw128<4>(r, jg * 16 + q4 * 4, 64)) =
               make_float4(out[q4 * 4], out[q4 * 4 + 1], out[q4 * 4 + 2], out[q4 * 4 + 3]);
       }
     }
     tc::fence_async_smem();
     cta_sync_tc();
 
-    // ---- P4: X = (I + N)^-1 by block forward substitution (16 x 16) ------
+    // ---- P4: X = (I + N)^-1; T = X diag(beta) -> bf16 -------------------
     {
       const float* N = reinterpret_cast<const float*>(smem + OFF_NMAT);
       float* X = reinterpret_cast<float*>(smem + OFF_XMAT);
       invert_unit_lower64(N, X, reinterpret_cast<float*>(smem + OFF_ZBUF), tid);
-      // T = X diag(beta) (lower triangle incl. diagonal) -> bf16 K-major [r][j]
-      {
-        const int r = tid >> 2, j0 = (tid & 3) * 16;
+      const int r = tid >> 3, j0 = (tid & 7) * 8;
+      uint32_t w[4];
 #pragma unroll
-        for (int h8 = 0; h8 < 2; ++h8) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 8; e += 2) {
-            const int j = j0 + h8 * 8 + e;
-            const float x0 = j <= r ? X[r * kLd + j] * s_beta[j] : 0.f;
-            const float x1 = j + 1 <= r ? X[r * kLd + j + 1] * s_beta[j + 1] : 0.f;
-            w[e >> 1] = pack_bf16x2(x0, x1);
-          }
-          *reinterpret_cast<uint4*>(smem + OFF_TM + tc::sw128<2>(r, j0 + h8 * 8, 64)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
-        }
+      for (int e = 0; e < 8; e += 2) {
+        const int j = j0 + e;
+        const float x0 = j <= r ? X[r * kLd + j] * s_beta[j] : 0.f;
+        const float x1 = j + 1 <= r ? X[r * kLd + j + 1] * s_beta[j + 1] : 0.f;
+        w[e >> 1] = pack_bf16x2(x0, x1);
       }
+      *reinterpret_cast<uint4*>(smem + OFF_TM + tc::sw128<2>(r, j0, 64)) =
+          make_uint4(w[0], w[1], w[2], w[3]);
     }
     tc::fence_async_smem();
     cta_sync_tc();
 
-    // ---- P5: W^T = (K e^g)^T T^T and U^T = V^T T^T (M=128, N=64, K=64) ----
+    // ---- P5: W^T = (K e^g)^T T^T and U^T = V^T T^T (M=128, N=64, K=64);
+    // meanwhile S0 -> bf16 tile and the decay of the fp32 state -------------
     if (tid == 0) {
       constexpr uint32_t idesc = tc::make_idesc(1, 1, 0, 128, 64);
 #pragma unroll
@@ -516,50 +514,41 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       }
       tc::mma_commit(mbar);
     }
+    {
+      const uint32_t tb = tmem + lane_off + TM_S + grp * 32;
+      float s[32];
+      tc::tmem_ld32(tb, s);
+      const int cb = grp * 32;
+#pragma unroll
+      for (int h8 = 0; h8 < 4; ++h8) {
+        uint32_t p[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) p[e] = pack_bf16x2(s[h8 * 8 + 2 * e], s[h8 * 8 + 2 * e + 1]);
+        *reinterpret_cast<uint4*>(smem + OFF_SB + tc::sw128<2>(m, cb + h8 * 8, 128)) =
+            make_uint4(p[0], p[1], p[2], p[3]);
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) s[i] *= s_gamma[cb + i];
+      tc::tmem_st16(tb, s);
+      tc::tmem_st16(tb + 16, s + 16);
+      tc::tmem_wait_st();
+    }
     ok = cta_wait(mbar, phase, 2);
     phase ^= 1;
     if (!ok) break;
-
-    // ---- P6: -W^T to shared memory; S0 -> bf16; decay of the fp32 state --
-    if (warp < 4) {
-      const int c = warp * 32 + lane;
-      const uint32_t tb = tmem + (static_cast<uint32_t>(warp * 32) << 16) + TM_W;
-#pragma unroll
-      for (int rg = 0; rg < 2; ++rg) {
-        float w[32];
-        tc::tmem_ld32(tb + rg * 32, w);
-#pragma unroll
-        for (int h8 = 0; h8 < 4; ++h8) {
-          uint32_t p[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            p[e] = pack_bf16x2(-w[h8 * 8 + 2 * e], -w[h8 * 8 + 2 * e + 1]);
-          *reinterpret_cast<uint4*>(smem + OFF_NW + tc::sw128<2>(c, rg * 32 + h8 * 8, 128)) =
-              make_uint4(p[0], p[1], p[2], p[3]);
-        }
-      }
-    }
     {
-      const uint32_t tb = tmem + lane_off + TM_S + half * 64;
+      // -W^T to shared memory: lane c holds W^T[c][r]; this warp takes r in [16 grp, +16).
+      float w[16];
+      tc::tmem_ld16(tmem + lane_off + TM_W + grp * 16, w);
 #pragma unroll
-      for (int cg = 0; cg < 2; ++cg) {
-        float s[32];
-        tc::tmem_ld32(tb + cg * 32, s);
-        const int cb = half * 64 + cg * 32;
+      for (int h8 = 0; h8 < 2; ++h8) {
+        uint32_t p[4];
 #pragma unroll
-        for (int h8 = 0; h8 < 4; ++h8) {
-          uint32_t p[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) p[e] = pack_bf16x2(s[h8 * 8 + 2 * e], s[h8 * 8 + 2 * e + 1]);
-          *reinterpret_cast<uint4*>(smem + OFF_SB + tc::sw128<2>(m, cb + h8 * 8, 128)) =
-              make_uint4(p[0], p[1], p[2], p[3]);
-        }
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[i] *= s_gamma[cb + i];
-        tc::tmem_st16(tb + cg * 32, s);
-        tc::tmem_st16(tb + cg * 32 + 16, s + 16);
+        for (int e = 0; e < 4; ++e)
+          p[e] = pack_bf16x2(-w[h8 * 8 + 2 * e], -w[h8 * 8 + 2 * e + 1]);
+        *reinterpret_cast<uint4*>(smem + OFF_NW + tc::sw128<2>(m, grp * 16 + h8 * 8, 128)) =
+            make_uint4(p[0], p[1], p[2], p[3]);
       }
-      tc::tmem_wait_st();
     }
     tc::fence_async_smem();
     cta_sync_tc();
@@ -584,7 +573,7 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     phase ^= 1;
     if (!ok) break;
 
-    // ---- P8: S^T += D^T K~ (tf32, A from TMEM); O^T += D^T M_qk^T ---------
+    // ---- P8: S^T += D^T K~ (tf32, A from TMEM, B K-major); O^T += D^T M_qk^T
     if (tid == 0) {
       constexpr uint32_t id_s = tc::make_idesc(2, 0, 0, 128, 128);
       constexpr uint32_t id_o = tc::make_idesc(2, 0, 0, 128, 64);
@@ -603,40 +592,20 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     ok = cta_wait(mbar, phase, 4);
     phase ^= 1;
     if (!ok) break;
-
-    // ---- P9: O to HBM (bf16), staged through shared memory ----------------
-    {
-      // The Q*e^g tile is dead once P7 completed: reuse it for O as [r][m].
-      __nv_bfloat16* otile = reinterpret_cast<__nv_bfloat16*>(smem + OFF_QT);
-      float ov[32];
-      tc::tmem_ld32(tmem + lane_off + TM_O + half * 32, ov);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) otile[(half * 32 + i) * DV + m] = __float2bfloat16_rn(ov[i]);
-      __syncthreads();
-#pragma unroll
-      for (int it = 0; it < 4; ++it) {
-        const int idx = it * kThreads + tid;
-        const int r = idx >> 4, c8 = idx & 15;
-        if (r < L)
-          *reinterpret_cast<uint4*>(o + ((size_t)(t0 + r) * H + head) * DV + c8 * 8) =
-              *reinterpret_cast<const uint4*>(otile + r * DV + c8 * 8);
-      }
-    }
-    cta_sync_tc();
   }
 
+  if (ok && n_chunks > 0) {
+    const long long t_last = t_begin + (long long)(n_chunks - 1) * C;
+    const int L_last = (int)(t_end - t_last);
+    store_output(tmem, lane_off, grp, m, smem + OFF_SB, o, t_last, L_last, H, head);
+  }
   if (ok && final_state) {
-    const uint32_t tb = tmem + lane_off + TM_S + half * 64;
+    float s[32];
+    tc::tmem_ld32(tmem + lane_off + TM_S + grp * 32, s);
 #pragma unroll
-    for (int cg = 0; cg < 4; ++cg) {
-      float s[16];
-      tc::tmem_ld16(tb + cg * 16, s);
-      tc::tmem_wait_ld();
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int c = half * 64 + cg * 16 + i;
-        final_state[state_off + (size_t)c * DV + m] = s[i];
-      }
+    for (int i = 0; i < 32; ++i) {
+      const int c = grp * 32 + i;
+      final_state[state_off + (size_t)c * DV + m] = s[i];
     }
   }
   if (!ok) {
