@@ -4,3 +4,4 @@
 #include "kda_decode.cu"
 #include "kda_recurrent.cu"
 #include "kda_chunk.cu"
+#include "kda_noalloc.cu"

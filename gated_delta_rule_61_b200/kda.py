@@ -22,7 +22,8 @@ KDA_F32, KDA_BF16 = 0, 1
 CHUNK_LOG_ALPHA_MIN = -10.0
 
 EXPORTS = ("kda_status_string", "kda_version", "kda_prefill_workspace_bytes",
-           "kda_prefill", "kda_decode_step", "kda_get_device_status")
+           "kda_prefill", "kda_decode_step", "kda_prefill_noalloc", "kda_get_device_status")
+NOALLOC_MAX_SEQS = 65536
 
 
 class KdaError(RuntimeError):
@@ -55,6 +56,8 @@ def lib():
     L.kda_prefill.restype = ctypes.c_int
     L.kda_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, ip, ip, ip, ip, ctypes.c_int, vp, vp]
     L.kda_decode_step.restype = ctypes.c_int
+    L.kda_prefill_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, i32p, ip, ip, ip, vp, fp, vp]
+    L.kda_prefill_noalloc.restype = ctypes.c_int
     L.kda_get_device_status.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int), vp]
     L.kda_get_device_status.restype = ctypes.c_int
     _lib = L
@@ -141,6 +144,46 @@ def prefill(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, *, chunk
         int(chunk), _ptr(o), _ptr(final_state), _ptr(workspace), ws_bytes, _stream(stream))
     if st != KDA_OK:
         raise KdaError(st, "kda_prefill")
+    return o, final_state
+
+
+def prefill_noalloc(q, k, v, log_alpha, beta, cu_seqlens, init_state=None, *,
+                    output_final_state=True, o=None, final_state=None, stream=None):
+    """Packed variable-length chunked prefill that allocates no device memory
+    inside the library (its scratch is a fixed array in libkda.so; see
+    kda_prefill_noalloc in include/kda.h for the limits and the sharing rule).
+    q, k, log_alpha [1, T, H, 128]; v [1, T, H, 128] (bf16); beta [1, T, H];
+    cu_seqlens int32 [N+1]; init_state [N, H, 128, 128] fp32 or None.
+    Returns (o, final_state). Output tensors are allocated here by torch
+    unless passed in; pass o and final_state to keep the call allocation-free."""
+    B, T, H, dk = q.shape
+    dev = q.device
+    n_seq = cu_seqlens.shape[0] - 1
+    if B != 1 or dk != 128 or v.shape[-1] != 128 or q.dtype != torch.bfloat16:
+        raise ValueError("prefill_noalloc takes packed bf16 inputs [1, T, H, 128]")
+    for t, name, shape, dtype in ((q, "q", (1, T, H, 128), torch.bfloat16),
+                                  (k, "k", (1, T, H, 128), torch.bfloat16),
+                                  (v, "v", (1, T, H, 128), torch.bfloat16),
+                                  (log_alpha, "log_alpha", (1, T, H, 128), torch.float32),
+                                  (beta, "beta", (1, T, H), torch.float32),
+                                  (cu_seqlens, "cu_seqlens", (n_seq + 1,), torch.int32)):
+        _check(t, name, shape, dtype, dev)
+    if init_state is not None:
+        _check(init_state, "init_state", (n_seq, H, 128, 128), torch.float32, dev)
+    if o is None:
+        o = torch.empty((1, T, H, 128), dtype=torch.bfloat16, device=dev)
+    else:
+        _check(o, "o", (1, T, H, 128), torch.bfloat16, dev)
+    if output_final_state and final_state is None:
+        final_state = torch.empty((n_seq, H, 128, 128), dtype=torch.float32, device=dev)
+    elif final_state is not None:
+        _check(final_state, "final_state", (n_seq, H, 128, 128), torch.float32, dev)
+    st = lib().kda_prefill_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(init_state),
+        _ptr(cu_seqlens), int(n_seq), int(T), int(H), _ptr(o), _ptr(final_state),
+        _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_prefill_noalloc")
     return o, final_state
 
 

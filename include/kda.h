@@ -61,6 +61,9 @@ typedef enum {
 /* Lower bound applied to log_alpha by the chunked prefill path. */
 #define KDA_CHUNK_LOG_ALPHA_MIN (-10.0f)
 
+/* Most sequences one kda_prefill_noalloc call accepts (its fixed scratch). */
+#define KDA_NOALLOC_MAX_SEQS 65536
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char *kda_status_string(kda_status status);
 
@@ -123,6 +126,36 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v,
                            const float *log_alpha, const float *beta,
                            float *state, int B, int H, int dk, int dv,
                            kda_dtype dtype, void *o, cudaStream_t stream);
+
+/*
+ * kda_prefill_noalloc -- the packed variable-length chunked prefill of
+ * kda_prefill (cu_seqlens given, bf16, dk = dv = 128, chunk = 64) for callers
+ * that cannot allocate device memory. The source pages have no counterpart:
+ * this is a library convenience. kda_prefill needs a caller-provided
+ * workspace for its per-call scratch (the longest-first order of the
+ * sequences); this variant keeps that scratch in a fixed device array inside
+ * the library instead, so a caller that may not call cudaMalloc can still run
+ * it: a plugin or hook that is handed device pointers but owns no allocator, a
+ * serving runtime whose device memory is already reserved by its own pool,
+ * or a latency-critical path where an allocation (and the synchronisation it
+ * can imply) is not acceptable.
+ * Inputs and outputs are still caller-owned device memory, with the shapes of
+ * kda_prefill's packed form: q, k, log_alpha [T, H, 128]; v, o [T, H, 128]
+ * (bf16); beta [T, H]; cu_seqlens int32 [n_seq + 1]; init_state and
+ * final_state [n_seq, H, 128, 128] fp32 or NULL.
+ * Limits: n_seq <= KDA_NOALLOC_MAX_SEQS, else KDA_ERR_UNSUPPORTED and
+ * nothing is launched. The fixed scratch (256 KiB per device, held until the
+ * process exits) is shared by every call on a device, so calls whose work
+ * overlaps on the GPU race on it; calls on one stream are ordered and safe.
+ * The first call on a device looks up the scratch's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture begins. Allocates nothing and calls no allocating routine.
+ */
+kda_status kda_prefill_noalloc(const void *q, const void *k, const void *v,
+                               const float *log_alpha, const float *beta,
+                               const float *init_state, const int32_t *cu_seqlens,
+                               int n_seq, int T, int H, void *o, float *final_state,
+                               cudaStream_t stream);
 
 /*
  * kda_get_device_status -- synchronise `stream` and return the sticky device
