@@ -33,6 +33,7 @@ sys.path.insert(0, ROOT)
 METRIC = "KDA prefill tokens/s & decode state GB/s (fraction of B200 roofline), 1 GPU"
 PREFILL = dict(B=4, T=8192, H=16, dk=128, dv=128, chunk=64, init_std=0.1)
 DECODE = dict(B=256, H=32, dk=128, dv=128, std=0.05)
+VARLEN = dict(H=32)
 BYTES_PER_HEAD_TOKEN = 3 * 256 + 512 + 4 + 256        # q,k,v + log_alpha + beta + o
 FLOPS_PER_HEAD_TOKEN = 6 * 128 * 128 + 2 * 64 * (3 * 128 + 2 * 128)   # dense tiles, C = 64
 PROFILE = os.path.join(ROOT, "profiles", "chunk64_prefill_b4_t8192_h16.txt")
@@ -300,6 +301,42 @@ def bench_ours(args):
                             "unit": "GB/s", "frac": gbs / world / hbm, "traffic": None,
                             "peak_kind": peak_kind}}
         del steps_in, S
+    # ---------------- packed variable-length prefill ----------------
+    var = None
+    if not args.no_varlen:
+        from gated_delta_rule_61_b200.inputs import varlen_lengths
+        lengths = varlen_lengths(64, 128, 32768, seed=0)
+        vin = prefill_inputs(1, 0, VARLEN["H"], 128, 128, dtype=torch.bfloat16, seed=2000 + rank,
+                             init_std=0.1, lengths=lengths, device=dev)
+        vo = torch.empty_like(vin["v"])
+        vs = torch.empty_like(vin["init_state"])
+        ws = torch.empty(kda.workspace_bytes(len(lengths), True), dtype=torch.uint8, device=dev)
+
+        def vstep():
+            kda.prefill(vin["q"], vin["k"], vin["v"], vin["log_alpha"], vin["beta"],
+                        init_state=vin["init_state"], cu_seqlens=vin["cu_seqlens"], chunk=64,
+                        o=vo, final_state=vs, workspace=ws, stream=stream)
+
+        vstep()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_v = 3
+        a.record(stream)
+        for _ in range(n_v):
+            vstep()
+        b.record(stream)
+        barrier(world)
+        vms = max_over_ranks(a.elapsed_time(b), world) / n_v
+        t_tot = sum(lengths)
+        vbytes = t_tot * VARLEN["H"] * BYTES_PER_HEAD_TOKEN + 2 * len(lengths) * VARLEN["H"] * 128 * 128 * 4
+        vgbs = vbytes / (vms * 1e-3) / 1e9
+        var = {"value": world * t_tot / (vms * 1e-3), "unit": "tokens/s", "ms_per_step": vms,
+               "workload": "KDA packed varlen prefill: 64 sequences log-uniform in [128, 32768] "
+                           "(%d tokens, longest %d), H=32, d=128, bf16, C=64" % (t_tot, max(lengths)),
+               "roofline": {"bound": "hbm", "achieved": vgbs, "peak": hbm, "unit": "GB/s",
+                            "frac": vgbs / hbm, "traffic": None, "peak_kind": peak_kind},
+               "gpu_launches_per_step": 2}
+        del vin, vo, vs
     clk.__exit__(None, None, None)
 
     # ---------------- end to end through the public API (host buffers) ----------------
@@ -355,7 +392,7 @@ def bench_ours(args):
                          "peak_kind": peak_kind, "kernel_ms": kernel_ms,
                          "tensor": {"achieved_tflops": tflops, "peak_tflops": bf16_tf,
                                     "frac": tflops / bf16_tf}},
-            "decode": dec, "e2e": e2e, "cpu_baseline": cpu,
+            "decode": dec, "varlen": var, "e2e": e2e, "cpu_baseline": cpu,
             "gpu_launches": args.steps, "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
@@ -373,6 +410,7 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-varlen", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--ref-budget", type=float, default=8.0)
