@@ -77,9 +77,9 @@ constexpr uint32_t OFF_XMAT = OFF_BG + 17408;  // X, fp32 [64][68]
 constexpr uint32_t OFF_ZBUF = OFF_BG + 34816;  // block products, fp32 [32][34]
 constexpr uint32_t OFF_NW = OFF_BG;            // after the solve: -W^T bf16 MN-major [c][r]
 constexpr uint32_t OFF_MISC = 188416;
-constexpr uint32_t MISC_GAMMA = 0, MISC_BETA = 512, MISC_TOT = 768, MISC_GF = 4864,
-                   MISC_GL = 8960, MISC_MBAR = 13056, MISC_TMEM = 13064;
-constexpr uint32_t kSmemBytes = OFF_MISC + 13072 + 1024;
+constexpr uint32_t MISC_GAMMA = 0, MISC_BETA = 512, MISC_GLAST = 768, MISC_PAIR = 1280,
+                   MISC_GF = 17664, MISC_GL = 19712, MISC_MBAR = 21760, MISC_TMEM = 21768;
+constexpr uint32_t kSmemBytes = OFF_MISC + 21776 + 1024;
 
 // Tensor-memory columns.
 constexpr uint32_t TM_S = 0, TM_D = 128, TM_O = 192, TM_G = 256, TM_W = 256;
@@ -87,6 +87,34 @@ constexpr uint32_t TM_S = 0, TM_D = 128, TM_O = 192, TM_G = 256, TM_W = 256;
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&p);
+}
+
+// 1/x for normal positive x by Newton-Raphson on the reciprocal (two steps
+// from an initial estimate read off the IEEE-754 exponent and mantissa bits,
+// the classic "magic constant" start): relative error below 3e-4, ample for
+// operands that are rounded to bf16 next. Runs on the FMA pipe, leaving the
+// exponential unit to the exponentials.
+__device__ __forceinline__ float rcp_newton(float x) {
+  float y = __int_as_float(0x7EF311C7 - __float_as_int(x));
+  y = y * fmaf(-x, y, 2.0f);
+  y = y * fmaf(-x, y, 2.0f);
+  return y;
+}
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+// Warp-level 16x8x8 tf32 MMA (fp32 accumulate), used for the 32 x 32 block
+// products of the triangular inverse.
+__device__ __forceinline__ void mma_16x8x8_tf32(float* d, const uint32_t* a, const uint32_t* b) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
 // Thread 0 spins (bounded) on the MMA barrier phase; the outcome is shared
@@ -155,37 +183,48 @@ __device__ __forceinline__ void invert_unit_lower64(const float* N, float* X, fl
     X[(b + rr) * kLd + a + cc] = -(x0 + x1);
     __syncthreads();
   }
-  // Level 3: Z = N[32:64, 0:32] X[0:32, 0:32];  X[32:64, 0:32] = -X[32:64, 32:64] Z.
-  {
-    const int r = t >> 4, c2 = (t & 15) * 2;
-    float z0 = 0.f, z1 = 0.f, y0 = 0.f, y1 = 0.f;
+  // Level 3: Z = N[32:64, 0:32] X[0:32, 0:32];  X[32:64, 0:32] = -X[32:64, 32:64] Z,
+  // as tf32 m16n8k8 MMAs: warps 0..7 each own one 16 x 8 tile of the 32 x 32 result.
+  const int warp = t >> 5, lane = t & 31, gid = lane >> 2, tig = lane & 3;
+  const int mt = (warp >> 2) & 1, nt = warp & 3;
+  if (warp < 8) {
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int kk = 0; kk < 32; kk += 2) {
-      const float n0 = N[(32 + r) * kLd + kk], n1 = N[(32 + r) * kLd + kk + 1];
-      const float2 xa = *reinterpret_cast<const float2*>(X + kk * kLd + c2);
-      const float2 xb = *reinterpret_cast<const float2*>(X + (kk + 1) * kLd + c2);
-      // X[0:32, 0:32] is lower triangular: entry (kk, c) is live for kk >= c.
-      z0 += n0 * (kk >= c2 ? xa.x : 0.f);
-      z1 += n0 * (kk >= c2 + 1 ? xa.y : 0.f);
-      y0 += n1 * (kk + 1 >= c2 ? xb.x : 0.f);
-      y1 += n1 * (kk + 1 >= c2 + 1 ? xb.y : 0.f);
+    for (int kt = 0; kt < 4; ++kt) {
+      if (kt < nt) continue;  // X[0:32,0:32] is lower triangular: these columns are zero
+      const int r0 = 32 + 16 * mt + gid, k0 = 8 * kt + tig;
+      const uint32_t a[4] = {to_tf32(N[r0 * kLd + k0]), to_tf32(N[(r0 + 8) * kLd + k0]),
+                             to_tf32(N[r0 * kLd + k0 + 4]), to_tf32(N[(r0 + 8) * kLd + k0 + 4])};
+      const int c = 8 * nt + gid;
+      const uint32_t b[2] = {to_tf32(k0 >= c ? X[k0 * kLd + c] : 0.f),
+                             to_tf32(k0 + 4 >= c ? X[(k0 + 4) * kLd + c] : 0.f)};
+      mma_16x8x8_tf32(d, a, b);
     }
-    *reinterpret_cast<float2*>(Z + r * 34 + c2) = make_float2(z0 + y0, z1 + y1);
-    __syncthreads();
-    float x0 = 0.f, x1 = 0.f, w0 = 0.f, w1 = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < 32; kk += 2) {
-      // X[32:64, 32:64] is lower triangular: (r, kk) is live for kk <= r.
-      const float d0 = kk <= r ? X[(32 + r) * kLd + 32 + kk] : 0.f;
-      const float d1 = kk + 1 <= r ? X[(32 + r) * kLd + 33 + kk] : 0.f;
-      const float2 za = *reinterpret_cast<const float2*>(Z + kk * 34 + c2);
-      const float2 zb = *reinterpret_cast<const float2*>(Z + (kk + 1) * 34 + c2);
-      x0 += d0 * za.x; x1 += d0 * za.y;
-      w0 += d1 * zb.x; w1 += d1 * zb.y;
-    }
-    *reinterpret_cast<float2*>(X + (32 + r) * kLd + c2) = make_float2(-(x0 + w0), -(x1 + w1));
-    __syncthreads();
+    const int zr = 16 * mt + gid, zc = 8 * nt + 2 * tig;
+    *reinterpret_cast<float2*>(Z + zr * 34 + zc) = make_float2(d[0], d[1]);
+    *reinterpret_cast<float2*>(Z + (zr + 8) * 34 + zc) = make_float2(d[2], d[3]);
   }
+  __syncthreads();
+  if (warp < 8) {
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int kt = 0; kt < 4; ++kt) {
+      if (kt > 2 * mt + 1) continue;  // X[32:64,32:64] is lower triangular
+      const int r0 = 16 * mt + gid, k0 = 8 * kt + tig;   // rows/cols within the block
+      const uint32_t a[4] = {
+          to_tf32(k0 <= r0 ? X[(32 + r0) * kLd + 32 + k0] : 0.f),
+          to_tf32(k0 <= r0 + 8 ? X[(40 + r0) * kLd + 32 + k0] : 0.f),
+          to_tf32(k0 + 4 <= r0 ? X[(32 + r0) * kLd + 36 + k0] : 0.f),
+          to_tf32(k0 + 4 <= r0 + 8 ? X[(40 + r0) * kLd + 36 + k0] : 0.f)};
+      const int c = 8 * nt + gid;
+      const uint32_t b[2] = {to_tf32(Z[k0 * 34 + c]), to_tf32(Z[(k0 + 4) * 34 + c])};
+      mma_16x8x8_tf32(d, a, b);
+    }
+    const int xr = 32 + 16 * mt + gid, xc = 8 * nt + 2 * tig;
+    *reinterpret_cast<float2*>(X + xr * kLd + xc) = make_float2(-d[0], -d[1]);
+    *reinterpret_cast<float2*>(X + (xr + 8) * kLd + xc) = make_float2(-d[2], -d[3]);
+  }
+  __syncthreads();
 }
 
 // O^T (lane m, column r) of one chunk -> bf16 [r][m] in shared memory ->
@@ -209,6 +248,28 @@ __device__ __forceinline__ void store_output(uint32_t tmem, uint32_t lane_off, i
   }
 }
 
+// Same as store_output, run by warps 8..15 only (two per lane quadrant, 32
+// output rows each), synchronised with a named barrier among those 256 threads.
+__device__ __forceinline__ void store_output_8w(uint32_t tmem, uint32_t lane_off, int half, int m,
+                                                uint8_t* stage, __nv_bfloat16* o, long long t0,
+                                                int L, int H, int head) {
+  __nv_bfloat16* otile = reinterpret_cast<__nv_bfloat16*>(stage);
+  float ov[32];
+  tc::tmem_ld32(tmem + lane_off + TM_O + half * 32, ov);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) otile[(half * 32 + i) * DV + m] = __float2bfloat16_rn(ov[i]);
+  asm volatile("bar.sync 1, 256;" ::: "memory");
+  const int t = threadIdx.x - 256;
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int idx = it * 256 + t;
+    const int r = idx >> 4, c8 = idx & 15;
+    if (r < L)
+      *reinterpret_cast<uint4*>(o + ((size_t)(t0 + r) * H + head) * DV + c8 * 8) =
+          *reinterpret_cast<const uint4*>(otile + r * DV + c8 * 8);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                const __nv_bfloat16* __restrict__ v, const float* __restrict__ log_alpha,
@@ -221,9 +282,8 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
   const uint32_t sbase = tc::smem_u32(smem);
   float* s_gamma = reinterpret_cast<float*>(smem + OFF_MISC + MISC_GAMMA);
   float* s_beta = reinterpret_cast<float*>(smem + OFF_MISC + MISC_BETA);
-  float* s_tot = reinterpret_cast<float*>(smem + OFF_MISC + MISC_TOT);   // [8][128]
-  float* s_gf = reinterpret_cast<float*>(smem + OFF_MISC + MISC_GF);     // [8][128]
-  float* s_gl = reinterpret_cast<float*>(smem + OFF_MISC + MISC_GL);     // [8][128]
+  float* s_gf = reinterpret_cast<float*>(smem + OFF_MISC + MISC_GF);     // [4][128]
+  float* s_gl = reinterpret_cast<float*>(smem + OFF_MISC + MISC_GL);     // [4][128]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC + MISC_TMEM);
   const uint32_t mbar = sbase + OFF_MISC + MISC_MBAR;
 
@@ -268,143 +328,188 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
 
   const long long len = t_end - t_begin;
   const int n_chunks = (int)((len + C - 1) / C);
-  // P1 mapping: channel pair (c0, c0 + 1), rows [8 rg, 8 rg + 8) of sub-chunk rg / 2.
-  const int pr = tid & 63, rg = tid >> 6, sub = rg >> 1, c0 = 2 * pr;
+  // P1 mapping: channel pair (c0, c0 + 1); row slot i = 2 a + e holds row
+  // 16 a + 2 rg + e, so every thread owns two rows of each 16-row sub-chunk
+  // (the per-sub-chunk work of the off-diagonal Gram factors is balanced).
+  const int pr = tid & 63, rg = tid >> 6, c0 = 2 * pr;
+  float* s_pair = reinterpret_cast<float*>(smem + OFF_MISC + MISC_PAIR);   // [32][128]
+  float* s_glast = reinterpret_cast<float*>(smem + OFF_MISC + MISC_GLAST);
+  // Inputs of the chunk about to be processed, loaded one chunk ahead.
+  float2 lr[8];
+  uint32_t kr[8], qr[8], vr[8];
+  float bt[8];
+  auto load_rows = [&](long long tc0, int Lc) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = 16 * (i >> 1) + 2 * rg + (i & 1);
+      lr[i] = make_float2(0.f, 0.f);
+      kr[i] = qr[i] = vr[i] = 0u;
+      bt[i] = 0.f;
+      if (r < Lc) {
+        const size_t tok = (size_t)(tc0 + r) * H + head;
+        lr[i] = __ldg(reinterpret_cast<const float2*>(log_alpha + tok * DK + c0));
+        kr[i] = __ldg(reinterpret_cast<const unsigned int*>(k + tok * DK + c0));
+        qr[i] = __ldg(reinterpret_cast<const unsigned int*>(q + tok * DK + c0));
+        vr[i] = __ldg(reinterpret_cast<const unsigned int*>(v + tok * DV + c0));
+        bt[i] = __ldg(beta + tok);
+      }
+    }
+  };
+  if (n_chunks > 0) load_rows(t_begin, (int)(len < C ? len : C));
 
   for (int n = 0; n < n_chunks; ++n) {
     const long long t0 = t_begin + (long long)n * C;
-    const int L = (int)((t_end - t0) < C ? (t_end - t0) : C);
 
     // ---- P1: cumulative gates and operand tiles --------------------------
+    // Cumulative sums: pair sums per (sub-chunk, rg) -> one exclusive scan
+    // over the 32 pairs per channel -> each thread adds its own rows.
     float g0[8], g1[8];
-    uint32_t kr[8], qr[8], vr[8];
-    float bt[8];
     {
-      float2 lr[8];
+      float l0[8], l1[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const int r = rg * 8 + i;
-        lr[i] = make_float2(0.f, 0.f);
-        kr[i] = qr[i] = vr[i] = 0u;
-        bt[i] = 0.f;
-        if (r < L) {
-          const size_t tok = (size_t)(t0 + r) * H + head;
-          lr[i] = __ldg(reinterpret_cast<const float2*>(log_alpha + tok * DK + c0));
-          kr[i] = __ldg(reinterpret_cast<const unsigned int*>(k + tok * DK + c0));
-          qr[i] = __ldg(reinterpret_cast<const unsigned int*>(q + tok * DK + c0));
-          vr[i] = __ldg(reinterpret_cast<const unsigned int*>(v + tok * DV + c0));
-          bt[i] = __ldg(beta + tok);
-        }
-      }
-      float run0 = 0.f, run1 = 0.f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        run0 += fmaxf(lr[i].x, kLogAlphaMin);
-        run1 += fmaxf(lr[i].y, kLogAlphaMin);
-        g0[i] = run0;
-        g1[i] = run1;
-      }
-      s_tot[rg * 128 + c0] = run0;
-      s_tot[rg * 128 + c0 + 1] = run1;
-    }
-    __syncthreads();
-    {
-      float off0 = 0.f, off1 = 0.f;
-      for (int b = 0; b < rg; ++b) {
-        off0 += s_tot[b * 128 + c0];
-        off1 += s_tot[b * 128 + c0 + 1];
+        l0[i] = fmaxf(lr[i].x, kLogAlphaMin);
+        l1[i] = fmaxf(lr[i].y, kLogAlphaMin);
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        g0[i] += off0;
-        g1[i] += off1;
-      }
-      s_gf[rg * 128 + c0] = g0[0];
-      s_gf[rg * 128 + c0 + 1] = g1[0];
-      s_gl[rg * 128 + c0] = g0[7];
-      s_gl[rg * 128 + c0 + 1] = g1[7];
-      if (rg == 7) {
-        s_gamma[c0] = __expf(g0[7]);
-        s_gamma[c0 + 1] = __expf(g1[7]);
+      for (int a = 0; a < 4; ++a) {
+        s_pair[(a * 8 + rg) * 128 + c0] = l0[2 * a] + l0[2 * a + 1];
+        s_pair[(a * 8 + rg) * 128 + c0 + 1] = l1[2 * a] + l1[2 * a + 1];
       }
       if (pr == 0) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) s_beta[rg * 8 + i] = bt[i];
+        for (int i = 0; i < 8; ++i) s_beta[16 * (i >> 1) + 2 * rg + (i & 1)] = bt[i];
+      }
+      __syncthreads();
+      if (tid < 128) {
+        float run = 0.f;
+#pragma unroll 8
+        for (int idx = 0; idx < 32; ++idx) {
+          const float x = s_pair[idx * 128 + tid];
+          s_pair[idx * 128 + tid] = run;
+          run += x;
+        }
+        s_glast[tid] = run;
+        s_gamma[tid] = __expf(run);
+      }
+      __syncthreads();
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        const float b0 = s_pair[(a * 8 + rg) * 128 + c0], b1 = s_pair[(a * 8 + rg) * 128 + c0 + 1];
+        g0[2 * a] = b0 + l0[2 * a];
+        g0[2 * a + 1] = g0[2 * a] + l0[2 * a + 1];
+        g1[2 * a] = b1 + l1[2 * a];
+        g1[2 * a + 1] = g1[2 * a] + l1[2 * a + 1];
+      }
+      if (rg == 0) {
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          s_gf[a * 128 + c0] = g0[2 * a];
+          s_gf[a * 128 + c0 + 1] = g1[2 * a];
+        }
+      }
+      if (rg == 7) {
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          s_gl[a * 128 + c0] = g0[2 * a + 1];
+          s_gl[a * 128 + c0 + 1] = g1[2 * a + 1];
+        }
       }
     }
     __syncthreads();
     {
-      // Sub-chunk midpoints m_a = (g at its first row + g at its last row) / 2.
+      // Sub-chunk midpoints m_a and the per-channel factors, from five
+      // exponentials per channel: e^{m_0}, e^{m_a - m_(a-1)} and e^{g_last - m_3};
+      // every other factor is a product of these (all at most 1).
       float mid0[4], mid1[4];
 #pragma unroll
       for (int a = 0; a < 4; ++a) {
-        mid0[a] = 0.5f * (s_gf[(2 * a) * 128 + c0] + s_gl[(2 * a + 1) * 128 + c0]);
-        mid1[a] = 0.5f * (s_gf[(2 * a) * 128 + c0 + 1] + s_gl[(2 * a + 1) * 128 + c0 + 1]);
+        mid0[a] = 0.5f * (s_gf[a * 128 + c0] + s_gl[a * 128 + c0]);
+        mid1[a] = 0.5f * (s_gf[a * 128 + c0 + 1] + s_gl[a * 128 + c0 + 1]);
       }
-      const float m0 = sub == 0 ? mid0[0] : sub == 1 ? mid0[1] : sub == 2 ? mid0[2] : mid0[3];
-      const float m1 = sub == 0 ? mid1[0] : sub == 1 ? mid1[1] : sub == 2 ? mid1[2] : mid1[3];
-      const float glast0 = s_gl[7 * 128 + c0], glast1 = s_gl[7 * 128 + c0 + 1];
-      const float em0 = __expf(m0), em1 = __expf(m1);
-      const float kt0 = __expf(glast0 - m0), kt1 = __expf(glast1 - m1);
-      float rho0[4], rho1[4];
+      const float gl0 = s_glast[c0], gl1 = s_glast[c0 + 1];
+      float dd0[4], dd1[4];   // dd[a] = e^{m_a - m_(a-1)}, a >= 1
+      dd0[0] = dd1[0] = 1.f;
 #pragma unroll
-      for (int ap = 0; ap < 4; ++ap) {
-        rho0[ap] = ap > sub ? __expf(mid0[ap] - m0) : 0.f;
-        rho1[ap] = ap > sub ? __expf(mid1[ap] - m1) : 0.f;
+      for (int a = 1; a < 4; ++a) {
+        dd0[a] = __expf(mid0[a] - mid0[a - 1]);
+        dd1[a] = __expf(mid1[a] - mid1[a - 1]);
       }
-      float kt_c0[8], kt_c1[8];
-      // Swizzled byte offsets of this thread's rows r = 8 rg + i: (r & 7) = i and
-      // (r >> 3) = rg, so only (chunk ^ i) varies at run time.
+      float em0[4], em1[4], kt0[4], kt1[4];
+      em0[0] = __expf(mid0[0]);
+      em1[0] = __expf(mid1[0]);
+      kt0[3] = __expf(gl0 - mid0[3]);
+      kt1[3] = __expf(gl1 - mid1[3]);
+#pragma unroll
+      for (int a = 1; a < 4; ++a) {
+        em0[a] = em0[a - 1] * dd0[a];
+        em1[a] = em1[a - 1] * dd1[a];
+      }
+#pragma unroll
+      for (int a = 2; a >= 0; --a) {
+        kt0[a] = kt0[a + 1] * dd0[a + 1];
+        kt1[a] = kt1[a + 1] * dd1[a + 1];
+      }
+      // Swizzled row offsets: r = 16 a + 2 rg + e, so (r >> 3) = 2 a + (rg >> 2)
+      // and (r & 7) = 2 (rg & 3) + e.
       const int xr = (c0 & 63) >> 3;
-      const uint32_t colb = (uint32_t)((c0 & 7) * 2) + (uint32_t)rg * 1024u;
+      const uint32_t rbase = (uint32_t)((rg >> 2) * 1024 + (rg & 3) * 256);
+      const uint32_t xo0 = (uint32_t)(xr ^ (2 * (rg & 3))) << 4;
+      const uint32_t xo1 = (uint32_t)(xr ^ (2 * (rg & 3) + 1)) << 4;
+      const uint32_t colb = (uint32_t)((c0 & 7) * 2) + rbase;
       const uint32_t sl = (uint32_t)(c0 >> 6);
       uint8_t* const pAGk = smem + OFF_AG + sl * 16384u + colb;
       uint8_t* const pBGe = smem + OFF_BG + sl * 20480u + colb;
       uint8_t* const pQT = smem + OFF_QT + sl * 8192u + colb;
       uint8_t* const pBK = smem + OFF_BK + sl * 8192u + colb;
       uint8_t* const pVV = smem + OFF_VV + sl * 8192u + colb;
+      float kt_c0[8], kt_c1[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const uint32_t ro = (uint32_t)(i * 128) + ((uint32_t)(xr ^ i) << 4);
+        const int a = i >> 1, e = i & 1;
+        const uint32_t ro = (uint32_t)(a * 2048 + e * 128) + (e ? xo1 : xo0);
         // bf16 pairs widen exactly: low half << 16, high half masked.
         const float k0 = __uint_as_float(kr[i] << 16), k1 = __uint_as_float(kr[i] & 0xffff0000u);
         const float q0 = __uint_as_float(qr[i] << 16), q1 = __uint_as_float(qr[i] & 0xffff0000u);
-        const float f0 = __expf(g0[i] - m0), f1 = __expf(g1[i] - m1);
-        const float fi0 = __expf(m0 - g0[i]), fi1 = __expf(m1 - g1[i]);
+        const float f0 = __expf(g0[i] - mid0[a]), f1 = __expf(g1[i] - mid1[a]);
+        const float fi0 = rcp_newton(f0), fi1 = rcp_newton(f1);
         *reinterpret_cast<uint32_t*>(pAGk + ro) = pack_bf16x2(k0 * f0, k1 * f1);
         *reinterpret_cast<uint32_t*>(pAGk + ro + 8192) = pack_bf16x2(q0 * f0, q1 * f1);
         const float e0 = k0 * fi0, e1 = k1 * fi1;
         *reinterpret_cast<uint32_t*>(pBGe + ro) = pack_bf16x2(e0, e1);
-        if (sub < 1)
-          *reinterpret_cast<uint32_t*>(pBGe + ro + 8192) = pack_bf16x2(e0 * rho0[1], e1 * rho1[1]);
-        if (sub < 2)
-          *reinterpret_cast<uint32_t*>(pBGe + ro + 10240) =
-              pack_bf16x2(e0 * rho0[2], e1 * rho1[2]);
-        if (sub < 3)
-          *reinterpret_cast<uint32_t*>(pBGe + ro + 14336) =
-              pack_bf16x2(e0 * rho0[3], e1 * rho1[3]);
-        const float eg0 = f0 * em0, eg1 = f1 * em1;
+        // R sets: row 64 + r (a < 1), 80 + r (a < 2), 112 + r (a < 3), scaled
+        // by e^{m_a' - m_a} = product of the dd factors in between.
+        if (a < 1)
+          *reinterpret_cast<uint32_t*>(pBGe + ro + 8192) =
+              pack_bf16x2(e0 * dd0[1], e1 * dd1[1]);
+        if (a < 2)
+          *reinterpret_cast<uint32_t*>(pBGe + ro + 10240) = pack_bf16x2(
+              e0 * (a == 0 ? dd0[1] * dd0[2] : dd0[2]), e1 * (a == 0 ? dd1[1] * dd1[2] : dd1[2]));
+        if (a < 3)
+          *reinterpret_cast<uint32_t*>(pBGe + ro + 14336) = pack_bf16x2(
+              e0 * (a == 0 ? dd0[1] * dd0[2] * dd0[3] : a == 1 ? dd0[2] * dd0[3] : dd0[3]),
+              e1 * (a == 0 ? dd1[1] * dd1[2] * dd1[3] : a == 1 ? dd1[2] * dd1[3] : dd1[3]));
+        const float eg0 = f0 * em0[a], eg1 = f1 * em1[a];
         *reinterpret_cast<uint32_t*>(pQT + ro) = pack_bf16x2(q0 * eg0, q1 * eg1);
         *reinterpret_cast<uint32_t*>(pBK + ro) = pack_bf16x2(k0 * eg0, k1 * eg1);
         *reinterpret_cast<uint32_t*>(pVV + ro) = vr[i];
-        kt_c0[i] = e0 * kt0;
-        kt_c1[i] = e1 * kt1;
+        kt_c0[i] = e0 * kt0[a];
+        kt_c1[i] = e1 * kt1[a];
       }
-      // K~ as a K-major tf32 operand [c][j]: 8 consecutive positions per channel.
+      // K~ as a K-major tf32 operand [c][j]: positions 16 a + 2 rg, +1 per channel.
 #pragma unroll
-      for (int q4 = 0; q4 < 2; ++q4) {
-        const int j = rg * 8 + q4 * 4;
-        *reinterpret_cast<float4*>(smem + OFF_KT + tc::sw128<4>(c0, j, 128)) =
-            make_float4(kt_c0[q4 * 4], kt_c0[q4 * 4 + 1], kt_c0[q4 * 4 + 2], kt_c0[q4 * 4 + 3]);
-        *reinterpret_cast<float4*>(smem + OFF_KT + tc::sw128<4>(c0 + 1, j, 128)) =
-            make_float4(kt_c1[q4 * 4], kt_c1[q4 * 4 + 1], kt_c1[q4 * 4 + 2], kt_c1[q4 * 4 + 3]);
+      for (int a = 0; a < 4; ++a) {
+        const int j = 16 * a + 2 * rg;
+        *reinterpret_cast<float2*>(smem + OFF_KT + tc::sw128<4>(c0, j, 128)) =
+            make_float2(kt_c0[2 * a], kt_c0[2 * a + 1]);
+        *reinterpret_cast<float2*>(smem + OFF_KT + tc::sw128<4>(c0 + 1, j, 128)) =
+            make_float2(kt_c1[2 * a], kt_c1[2 * a + 1]);
       }
     }
     tc::fence_async_smem();
     cta_sync_tc();
 
-    // ---- P2: Gram MMA (M=128, N=160, K=128); meanwhile the previous chunk's
-    // output goes to HBM (staged in the S0 bf16 tile, dead until P5) --------
+    // ---- P2: Gram MMA (M=128, N=160, K=128) --------------------------------
     if (tid == 0) {
       constexpr uint32_t idesc = tc::make_idesc(1, 0, 0, 128, 160);
 #pragma unroll
@@ -417,7 +522,6 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       }
       tc::mma_commit(mbar);
     }
-    if (n > 0) store_output(tmem, lane_off, grp, m, smem + OFF_SB, o, t0 - C, C, H, head);
     if (n + 1 < n_chunks) {  // warm L2 with the next chunk's rows
       const long long t1 = t0 + C;
       const int row = tid >> 3, part = tid & 7;
@@ -484,6 +588,11 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     {
       const float* N = reinterpret_cast<const float*>(smem + OFF_NMAT);
       float* X = reinterpret_cast<float*>(smem + OFF_XMAT);
+      // Meanwhile warps 8..15 move the previous chunk's output to HBM (staged
+      // in the S0 bf16 tile, which is dead until P5).
+      if (n > 0 && warp >= 8)
+        store_output_8w(tmem, lane_off, (warp >> 2) & 1, m, smem + OFF_SB, o, t0 - C, C, H,
+                        head);
       invert_unit_lower64(N, X, reinterpret_cast<float*>(smem + OFF_ZBUF), tid);
       const int r = tid >> 3, j0 = (tid & 7) * 8;
       uint32_t w[4];
@@ -532,6 +641,12 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       tc::tmem_st16(tb, s);
       tc::tmem_st16(tb + 16, s + 16);
       tc::tmem_wait_st();
+    }
+    // This chunk's inputs are consumed: load the next chunk's now, so the
+    // loads are in flight during the state MMAs.
+    if (n + 1 < n_chunks) {
+      const long long t1 = t0 + C;
+      load_rows(t1, (int)((t_end - t1) < C ? (t_end - t1) : C));
     }
     ok = cta_wait(mbar, phase, 2);
     phase ^= 1;
