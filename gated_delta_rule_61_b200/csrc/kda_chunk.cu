@@ -36,7 +36,11 @@
 // and the state itself stays fp32 in tensor memory for the whole sequence.
 //
 // Layout. One CTA (512 threads = 16 warps) per (sequence, head) chain,
-// walking its chunks in order. Warp w reaches tensor-memory lanes
+// walking its chunks in order; or, when chains are few, a cluster of two CTAs
+// per chain that take alternate chunks: each CTA prepares its own chunks (the
+// state-independent work, most of the time) in parallel with its partner, and
+// the fp32 state moves to the partner through the chain's final_state slot
+// (L2) after each chunk's state update. Warp w reaches tensor-memory lanes
 // [32 (w % 4), +32); the four warps sharing a lane quadrant split the columns.
 // Tensor memory (512 columns, lanes = dv index m for the state-sized
 // accumulators):
@@ -78,8 +82,14 @@ constexpr uint32_t OFF_ZBUF = OFF_BG + 34816;  // block products, fp32 [32][34]
 constexpr uint32_t OFF_NW = OFF_BG;            // after the solve: -W^T bf16 MN-major [c][r]
 constexpr uint32_t OFF_MISC = 188416;
 constexpr uint32_t MISC_GAMMA = 0, MISC_BETA = 512, MISC_GLAST = 768, MISC_PAIR = 1280,
-                   MISC_GF = 17664, MISC_GL = 19712, MISC_MBAR = 21760, MISC_TMEM = 21768;
-constexpr uint32_t kSmemBytes = OFF_MISC + 21776 + 1024;
+                   MISC_GF = 17664, MISC_GL = 19712, MISC_MBAR = 21760, MISC_FULL = 21776,
+                   MISC_TMEM = 21784;
+constexpr uint32_t kSmemBytes = OFF_MISC + 21792 + 1024;
+// State hand-over between the two CTAs of a pair goes through the chain's
+// final_state slot in global memory (64 KiB, L2-resident): the two CTAs write
+// and read it strictly in turn (A writes S_n, B reads it, B writes S_n+1,
+// A reads it, ...), so one arrive on the reader's mbarrier per hand-over is
+// the only synchronisation needed.
 
 // Tensor-memory columns.
 constexpr uint32_t TM_S = 0, TM_D = 128, TM_O = 192, TM_G = 256, TM_W = 256;
@@ -270,12 +280,13 @@ __device__ __forceinline__ void store_output_8w(uint32_t tmem, uint32_t lane_off
   }
 }
 
+template <bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                const __nv_bfloat16* __restrict__ v, const float* __restrict__ log_alpha,
-               const float* __restrict__ beta, const float* __restrict__ init_state,
+               const float* __restrict__ beta, const float* init_state,
                const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ order,
-               int T, int H, __nv_bfloat16* __restrict__ o, float* __restrict__ final_state) {
+               int T, int H, __nv_bfloat16* __restrict__ o, float* final_state) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -288,7 +299,9 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
   const uint32_t mbar = sbase + OFF_MISC + MISC_MBAR;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int chain = blockIdx.x;
+  const int rank = kPair ? (int)tc::cluster_ctarank() : 0;
+  const int step = kPair ? 2 : 1;
+  const int chain = kPair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int seq = order ? order[chain / H] : chain / H;
   const int head = chain % H;
   long long t_begin, t_end;
@@ -298,13 +311,16 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     tc::tmem_alloc(tc::smem_u32(tmem_slot), 512);
     tc::tmem_relinquish();
   }
+  const uint32_t mbar_full = sbase + OFF_MISC + MISC_FULL;     // partner's state is in L2
   if (tid == 0) {
     tc::mbar_init(mbar, 1);
+    if (kPair) tc::mbar_init(mbar_full, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   cta_sync_tc();
+  if (kPair) tc::cluster_sync();   // partner's barriers exist before any remote arrive
   const uint32_t tmem = *tmem_slot;
-  uint32_t phase = 0;
+  uint32_t phase = 0, full_phase = 0;
   bool ok = true;
 
   const int quad = warp & 3, grp = warp >> 2;
@@ -313,7 +329,8 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
   const size_t state_off = ((size_t)seq * H + head) * DK * DV;
 
   // Initial state: S^T[m][c] = S0[c][m]; this warp covers columns [32 grp, +32).
-  {
+  // (With a pair, rank 1 receives its first state from rank 0.)
+  if (rank == 0) {
     float vals[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
@@ -355,9 +372,12 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       }
     }
   };
-  if (n_chunks > 0) load_rows(t_begin, (int)(len < C ? len : C));
+  if (rank < n_chunks) {
+    const long long tf = t_begin + (long long)rank * C;
+    load_rows(tf, (int)((t_end - tf) < C ? (t_end - tf) : C));
+  }
 
-  for (int n = 0; n < n_chunks; ++n) {
+  for (int n = rank; n < n_chunks; n += step) {
     const long long t0 = t_begin + (long long)n * C;
 
     // ---- P1: cumulative gates and operand tiles --------------------------
@@ -522,8 +542,8 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       }
       tc::mma_commit(mbar);
     }
-    if (n + 1 < n_chunks) {  // warm L2 with the next chunk's rows
-      const long long t1 = t0 + C;
+    if (n + step < n_chunks) {  // warm L2 with this CTA's next chunk
+      const long long t1 = t0 + (long long)step * C;
       const int row = tid >> 3, part = tid & 7;
       if (t1 + row < t_end) {
         const size_t tok = (size_t)(t1 + row) * H + head;
@@ -590,9 +610,9 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       float* X = reinterpret_cast<float*>(smem + OFF_XMAT);
       // Meanwhile warps 8..15 move the previous chunk's output to HBM (staged
       // in the S0 bf16 tile, which is dead until P5).
-      if (n > 0 && warp >= 8)
-        store_output_8w(tmem, lane_off, (warp >> 2) & 1, m, smem + OFF_SB, o, t0 - C, C, H,
-                        head);
+      if (n >= step && warp >= 8)
+        store_output_8w(tmem, lane_off, (warp >> 2) & 1, m, smem + OFF_SB, o,
+                        t0 - (long long)step * C, C, H, head);
       invert_unit_lower64(N, X, reinterpret_cast<float*>(smem + OFF_ZBUF), tid);
       const int r = tid >> 3, j0 = (tid & 7) * 8;
       uint32_t w[4];
@@ -623,7 +643,8 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       }
       tc::mma_commit(mbar);
     }
-    {
+    const bool receive = kPair && n > 0;
+    if (!receive) {
       const uint32_t tb = tmem + lane_off + TM_S + grp * 32;
       float s[32];
       tc::tmem_ld32(tb, s);
@@ -644,8 +665,8 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     }
     // This chunk's inputs are consumed: load the next chunk's now, so the
     // loads are in flight during the state MMAs.
-    if (n + 1 < n_chunks) {
-      const long long t1 = t0 + C;
+    if (n + step < n_chunks) {
+      const long long t1 = t0 + (long long)step * C;
       load_rows(t1, (int)((t_end - t1) < C ? (t_end - t1) : C));
     }
     ok = cta_wait(mbar, phase, 2);
@@ -664,6 +685,35 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         *reinterpret_cast<uint4*>(smem + OFF_NW + tc::sw128<2>(m, grp * 16 + h8 * 8, 128)) =
             make_uint4(p[0], p[1], p[2], p[3]);
       }
+    }
+    if (receive) {
+      // The partner wrote this chunk's entering state to the final_state slot.
+      int fail = tc::mbar_wait_cluster_bounded(mbar_full, full_phase, kMaxWaitNs) ? 0 : 1;
+      full_phase ^= 1;
+      fail = __syncthreads_or(fail);
+      if (fail) {
+        if (tid == 0) report_timeout(5);
+        ok = false;
+        break;
+      }
+      float s[32];
+      const int cb = grp * 32;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) s[i] = __ldcg(final_state + state_off + (size_t)(cb + i) * DV + m);
+#pragma unroll
+      for (int h8 = 0; h8 < 4; ++h8) {
+        uint32_t p[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) p[e] = pack_bf16x2(s[h8 * 8 + 2 * e], s[h8 * 8 + 2 * e + 1]);
+        *reinterpret_cast<uint4*>(smem + OFF_SB + tc::sw128<2>(m, cb + h8 * 8, 128)) =
+            make_uint4(p[0], p[1], p[2], p[3]);
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) s[i] *= s_gamma[cb + i];
+      const uint32_t tb = tmem + lane_off + TM_S + grp * 32;
+      tc::tmem_st16(tb, s);
+      tc::tmem_st16(tb + 16, s + 16);
+      tc::tmem_wait_st();
     }
     tc::fence_async_smem();
     cta_sync_tc();
@@ -707,14 +757,28 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     ok = cta_wait(mbar, phase, 4);
     phase ^= 1;
     if (!ok) break;
+
+    if (kPair && n + 1 < n_chunks) {
+      // Hand the state to the partner, which takes chunk n + 1.
+      float s[32];
+      tc::tmem_ld32(tmem + lane_off + TM_S + grp * 32, s);
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        __stcg(final_state + state_off + (size_t)(grp * 32 + i) * DV + m, s[i]);
+      asm volatile("fence.acq_rel.cluster;" ::: "memory");
+      __syncthreads();
+      if (tid == 0) tc::mbar_remote_arrive(tc::mapa_shared(mbar_full, (uint32_t)(rank ^ 1)));
+    }
   }
 
-  if (ok && n_chunks > 0) {
-    const long long t_last = t_begin + (long long)(n_chunks - 1) * C;
-    const int L_last = (int)(t_end - t_last);
+  if (ok && n_chunks > rank) {
+    const int n_mine = rank + step * ((n_chunks - 1 - rank) / step);   // this CTA's last chunk
+    const long long t_last = t_begin + (long long)n_mine * C;
+    const int L_last = (int)((t_end - t_last) < C ? (t_end - t_last) : C);
     store_output(tmem, lane_off, grp, m, smem + OFF_SB, o, t_last, L_last, H, head);
   }
-  if (ok && final_state) {
+  const bool owns_final = n_chunks > 0 ? ((n_chunks - 1) % step == rank) : rank == 0;
+  if (ok && final_state && owns_final) {
     float s[32];
     tc::tmem_ld32(tmem + lane_off + TM_S + grp * 32, s);
 #pragma unroll
@@ -729,6 +793,7 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     if (tid == 0) tc::mbar_wait_bounded(mbar, phase ^ 1, kMaxWaitNs);
   }
   cta_sync_tc();
+  if (kPair) tc::cluster_sync();   // no remote traffic targets this CTA past this point
   if (warp == 0) tc::tmem_dealloc(tmem, 512);
 }
 
@@ -760,9 +825,19 @@ cudaError_t launch_chunk64(const void* q, const void* k, const void* v, const fl
                            cudaStream_t stream) {
   using namespace chunk64;
   static bool attr_set = false;
+  static int n_sm = 0;
   if (!attr_set) {
-    const cudaError_t e = cudaFuncSetAttribute(
-        chunk64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(chunk64_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(chunk64_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    int dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -775,9 +850,32 @@ cudaError_t launch_chunk64(const void* q, const void* k, const void* v, const fl
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  chunk64_kernel<<<(unsigned)((long long)n_seq * H), kThreads, kSmemBytes, stream>>>(
-      (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, la, beta, s0,
-      cu, cu ? order : nullptr, T, H, (__nv_bfloat16*)o, sT);
+  const long long chains = (long long)n_seq * H;
+  const __nv_bfloat16* qb = (const __nv_bfloat16*)q;
+  const __nv_bfloat16* kb = (const __nv_bfloat16*)k;
+  const __nv_bfloat16* vb = (const __nv_bfloat16*)v;
+  const int32_t* ord = cu ? order : nullptr;
+  __nv_bfloat16* ob = (__nv_bfloat16*)o;
+  if (sT && 2 * chains <= n_sm) {
+    // Few chains: two CTAs per chain (alternate chunks), all in one wave; the
+    // state passes between them through the final_state slot.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * chains));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, chunk64_kernel<true>, qb, kb, vb, la, beta, s0, cu, ord, T,
+                              H, ob, sT);
+  }
+  chunk64_kernel<false><<<(unsigned)chains, kThreads, kSmemBytes, stream>>>(
+      qb, kb, vb, la, beta, s0, cu, ord, T, H, ob, sT);
   return cudaGetLastError();
 }
 
