@@ -36,11 +36,11 @@
 // and the state itself stays fp32 in tensor memory for the whole sequence.
 //
 // Layout. One CTA (512 threads = 16 warps) per (sequence, head) chain,
-// walking its chunks in order; or, when chains are few, a cluster of two CTAs
-// per chain that take alternate chunks: each CTA prepares its own chunks (the
-// state-independent work, most of the time) in parallel with its partner, and
-// the fp32 state moves to the partner through the chain's final_state slot
-// (L2) after each chunk's state update. Warp w reaches tensor-memory lanes
+// walking its chunks in order; or, when chains are few, a cluster of R = 2 or
+// 4 CTAs per chain that take chunks round-robin: each CTA prepares its own
+// chunks (the state-independent work, most of the time) in parallel with the
+// others, and the fp32 state moves to the next CTA through the chain's
+// final_state slot (L2) after each chunk's state update. Warp w reaches tensor-memory lanes
 // [32 (w % 4), +32); the four warps sharing a lane quadrant split the columns.
 // Tensor memory (512 columns, lanes = dv index m for the state-sized
 // accumulators):
@@ -85,11 +85,11 @@ constexpr uint32_t MISC_GAMMA = 0, MISC_BETA = 512, MISC_GLAST = 768, MISC_PAIR 
                    MISC_GF = 17664, MISC_GL = 19712, MISC_MBAR = 21760, MISC_FULL = 21776,
                    MISC_TMEM = 21784;
 constexpr uint32_t kSmemBytes = OFF_MISC + 21792 + 1024;
-// State hand-over between the two CTAs of a pair goes through the chain's
-// final_state slot in global memory (64 KiB, L2-resident): the two CTAs write
-// and read it strictly in turn (A writes S_n, B reads it, B writes S_n+1,
-// A reads it, ...), so one arrive on the reader's mbarrier per hand-over is
-// the only synchronisation needed.
+// State hand-over between the CTAs of a chain's cluster goes through the
+// chain's final_state slot in global memory (64 KiB, L2-resident): it is
+// written and read strictly in turn (CTA r writes S_n+1 after reading S_n;
+// CTA r+1 reads it before writing S_n+2), so one arrive on the reader's
+// mbarrier per hand-over is the only synchronisation needed.
 
 // Tensor-memory columns.
 constexpr uint32_t TM_S = 0, TM_D = 128, TM_O = 192, TM_G = 256, TM_W = 256;
@@ -280,7 +280,7 @@ __device__ __forceinline__ void store_output_8w(uint32_t tmem, uint32_t lane_off
   }
 }
 
-template <bool kPair>
+template <int kRing>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                const __nv_bfloat16* __restrict__ v, const float* __restrict__ log_alpha,
@@ -299,9 +299,10 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
   const uint32_t mbar = sbase + OFF_MISC + MISC_MBAR;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  constexpr bool kPair = kRing > 1;
   const int rank = kPair ? (int)tc::cluster_ctarank() : 0;
-  const int step = kPair ? 2 : 1;
-  const int chain = kPair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int step = kRing;
+  const int chain = (int)blockIdx.x / kRing;
   const int seq = order ? order[chain / H] : chain / H;
   const int head = chain % H;
   long long t_begin, t_end;
@@ -759,7 +760,7 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     if (!ok) break;
 
     if (kPair && n + 1 < n_chunks) {
-      // Hand the state to the partner, which takes chunk n + 1.
+      // Hand the state to the next CTA of the ring, which takes chunk n + 1.
       float s[32];
       tc::tmem_ld32(tmem + lane_off + TM_S + grp * 32, s);
 #pragma unroll
@@ -767,7 +768,8 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         __stcg(final_state + state_off + (size_t)(grp * 32 + i) * DV + m, s[i]);
       asm volatile("fence.acq_rel.cluster;" ::: "memory");
       __syncthreads();
-      if (tid == 0) tc::mbar_remote_arrive(tc::mapa_shared(mbar_full, (uint32_t)(rank ^ 1)));
+      if (tid == 0)
+        tc::mbar_remote_arrive(tc::mapa_shared(mbar_full, (uint32_t)((rank + 1) % kRing)));
     }
   }
 
@@ -827,11 +829,14 @@ cudaError_t launch_chunk64(const void* q, const void* k, const void* v, const fl
   static bool attr_set = false;
   static int n_sm = 0;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(chunk64_kernel<false>,
+    cudaError_t e = cudaFuncSetAttribute(chunk64_kernel<1>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(chunk64_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(chunk64_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(chunk64_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     int dev = 0;
@@ -857,24 +862,28 @@ cudaError_t launch_chunk64(const void* q, const void* k, const void* v, const fl
   const int32_t* ord = cu ? order : nullptr;
   __nv_bfloat16* ob = (__nv_bfloat16*)o;
   if (sT && 2 * chains <= n_sm) {
-    // Few chains: two CTAs per chain (alternate chunks), all in one wave; the
-    // state passes between them through the final_state slot.
+    // Few chains: R = 4 or 2 CTAs per chain (chunks round-robin), all in one
+    // wave; the state passes between them through the final_state slot.
+    const int ring = 4 * chains <= n_sm ? 4 : 2;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(2 * chains));
+    cfg.gridDim = dim3((unsigned)(ring * chains));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.x = (unsigned)ring;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, chunk64_kernel<true>, qb, kb, vb, la, beta, s0, cu, ord, T,
-                              H, ob, sT);
+    if (ring == 4)
+      return cudaLaunchKernelEx(&cfg, chunk64_kernel<4>, qb, kb, vb, la, beta, s0, cu, ord, T,
+                                H, ob, sT);
+    return cudaLaunchKernelEx(&cfg, chunk64_kernel<2>, qb, kb, vb, la, beta, s0, cu, ord, T, H,
+                              ob, sT);
   }
-  chunk64_kernel<false><<<(unsigned)chains, kThreads, kSmemBytes, stream>>>(
+  chunk64_kernel<1><<<(unsigned)chains, kThreads, kSmemBytes, stream>>>(
       qb, kb, vb, la, beta, s0, cu, ord, T, H, ob, sT);
   return cudaGetLastError();
 }
