@@ -89,7 +89,12 @@ constexpr uint32_t kSmemBytes = OFF_MISC + 21792 + 1024;
 // chain's final_state slot in global memory (64 KiB, L2-resident): it is
 // written and read strictly in turn (CTA r writes S_n+1 after reading S_n;
 // CTA r+1 reads it before writing S_n+2), so one arrive on the reader's
-// mbarrier per hand-over is the only synchronisation needed.
+// mbarrier per hand-over is the only synchronisation needed. While it
+// carries a hand-over the slot holds S^T in 16-byte chunks ordered
+// (column group c / 4, row m), so each warp moves 512 contiguous bytes per
+// access; the owner of the last chunk writes the final state in its own
+// [dk][dv] layout.
+__device__ __forceinline__ size_t xfer_chunk(int m, int c4) { return (size_t)c4 * 128 + m; }
 
 // Tensor-memory columns.
 constexpr uint32_t TM_S = 0, TM_D = 128, TM_O = 192, TM_G = 256, TM_W = 256;
@@ -323,6 +328,18 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
   const uint32_t tmem = *tmem_slot;
   uint32_t phase = 0, full_phase = 0;
   bool ok = true;
+  bool signal_pending = false;   // a state hand-over written but not yet announced
+  // Announce a written hand-over to the next CTA of the ring (thread 0, after
+  // a CTA barrier that follows every thread's stores).
+  auto flush_signal = [&]() {
+    if (kPair && signal_pending) {
+      if (tid == 0) {
+        asm volatile("fence.acq_rel.cluster;" ::: "memory");
+        tc::mbar_remote_arrive(tc::mapa_shared(mbar_full, (uint32_t)((rank + 1) % kRing)));
+      }
+      signal_pending = false;
+    }
+  };
 
   const int quad = warp & 3, grp = warp >> 2;
   const int m = quad * 32 + lane;
@@ -414,6 +431,7 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         s_gamma[tid] = __expf(run);
       }
       __syncthreads();
+      flush_signal();
 #pragma unroll
       for (int a = 0; a < 4; ++a) {
         const float b0 = s_pair[(a * 8 + rg) * 128 + c0], b1 = s_pair[(a * 8 + rg) * 128 + c0 + 1];
@@ -699,8 +717,12 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       }
       float s[32];
       const int cb = grp * 32;
+      const float4* slot = reinterpret_cast<const float4*>(final_state + state_off);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) s[i] = __ldcg(final_state + state_off + (size_t)(cb + i) * DV + m);
+      for (int v4 = 0; v4 < 8; ++v4) {
+        const float4 x = __ldcg(slot + xfer_chunk(m, cb / 4 + v4));
+        s[4 * v4] = x.x; s[4 * v4 + 1] = x.y; s[4 * v4 + 2] = x.z; s[4 * v4 + 3] = x.w;
+      }
 #pragma unroll
       for (int h8 = 0; h8 < 4; ++h8) {
         uint32_t p[4];
@@ -763,16 +785,26 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       // Hand the state to the next CTA of the ring, which takes chunk n + 1.
       float s[32];
       tc::tmem_ld32(tmem + lane_off + TM_S + grp * 32, s);
+      float4* slot = reinterpret_cast<float4*>(final_state + state_off);
 #pragma unroll
-      for (int i = 0; i < 32; ++i)
-        __stcg(final_state + state_off + (size_t)(grp * 32 + i) * DV + m, s[i]);
-      asm volatile("fence.acq_rel.cluster;" ::: "memory");
-      __syncthreads();
-      if (tid == 0)
-        tc::mbar_remote_arrive(tc::mapa_shared(mbar_full, (uint32_t)((rank + 1) % kRing)));
+      for (int v4 = 0; v4 < 8; ++v4)
+        __stcg(slot + xfer_chunk(m, grp * 8 + v4),
+               make_float4(s[4 * v4], s[4 * v4 + 1], s[4 * v4 + 2], s[4 * v4 + 3]));
+      // With two CTAs per chain the partner is still busy with its own chunk
+      // preparation, so it is told later (signal_pending: after a CTA barrier
+      // in the next chunk, once the stores have landed and the release fence
+      // is cheap). With four, the hand-over is on the critical path: tell it
+      // now.
+      signal_pending = true;
+      if (kRing > 2) {
+        __syncthreads();
+        flush_signal();
+      }
     }
   }
 
+  __syncthreads();
+  flush_signal();
   if (ok && n_chunks > rank) {
     const int n_mine = rank + step * ((n_chunks - 1 - rank) / step);   // this CTA's last chunk
     const long long t_last = t_begin + (long long)n_mine * C;
