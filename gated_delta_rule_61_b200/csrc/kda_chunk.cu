@@ -211,8 +211,8 @@ __device__ __forceinline__ void invert_unit_lower64(const float* N, float* X, fl
       const uint32_t a[4] = {to_tf32(N[r0 * kLd + k0]), to_tf32(N[(r0 + 8) * kLd + k0]),
                              to_tf32(N[r0 * kLd + k0 + 4]), to_tf32(N[(r0 + 8) * kLd + k0 + 4])};
       const int c = 8 * nt + gid;
-      const uint32_t b[2] = {to_tf32(k0 >= c ? X[k0 * kLd + c] : 0.f),
-                             to_tf32(k0 + 4 >= c ? X[(k0 + 4) * kLd + c] : 0.f)};
+      const float x0 = X[k0 * kLd + c], x1 = X[(k0 + 4) * kLd + c];
+      const uint32_t b[2] = {to_tf32(k0 >= c ? x0 : 0.f), to_tf32(k0 + 4 >= c ? x1 : 0.f)};
       mma_16x8x8_tf32(d, a, b);
     }
     const int zr = 16 * mt + gid, zc = 8 * nt + 2 * tig;
@@ -226,11 +226,11 @@ __device__ __forceinline__ void invert_unit_lower64(const float* N, float* X, fl
     for (int kt = 0; kt < 4; ++kt) {
       if (kt > 2 * mt + 1) continue;  // X[32:64,32:64] is lower triangular
       const int r0 = 16 * mt + gid, k0 = 8 * kt + tig;   // rows/cols within the block
-      const uint32_t a[4] = {
-          to_tf32(k0 <= r0 ? X[(32 + r0) * kLd + 32 + k0] : 0.f),
-          to_tf32(k0 <= r0 + 8 ? X[(40 + r0) * kLd + 32 + k0] : 0.f),
-          to_tf32(k0 + 4 <= r0 ? X[(32 + r0) * kLd + 36 + k0] : 0.f),
-          to_tf32(k0 + 4 <= r0 + 8 ? X[(40 + r0) * kLd + 36 + k0] : 0.f)};
+      const float y0 = X[(32 + r0) * kLd + 32 + k0], y1 = X[(40 + r0) * kLd + 32 + k0];
+      const float y2 = X[(32 + r0) * kLd + 36 + k0], y3 = X[(40 + r0) * kLd + 36 + k0];
+      const uint32_t a[4] = {to_tf32(k0 <= r0 ? y0 : 0.f), to_tf32(k0 <= r0 + 8 ? y1 : 0.f),
+                             to_tf32(k0 + 4 <= r0 ? y2 : 0.f),
+                             to_tf32(k0 + 4 <= r0 + 8 ? y3 : 0.f)};
       const int c = 8 * nt + gid;
       const uint32_t b[2] = {to_tf32(Z[k0 * 34 + c]), to_tf32(Z[(k0 + 4) * 34 + c])};
       mma_16x8x8_tf32(d, a, b);
@@ -594,16 +594,17 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       float vv[64];
       tc::tmem_ld16x4(tb + 16 * jg, tb + (jg == 0 ? c_r1 : 16 * jg),
                       tb + (jg <= 1 ? c_r2 : 16 * jg), tb + (jg <= 2 ? c_r3 : 16 * jg), vv);
+      // Branch-free selection (the row's sub-chunk ar differs between lanes):
+      // column block jg < ar comes from R_ar, jg == ar from the diagonal set
+      // under the causal mask, jg > ar is zero.
+      const bool from_r = jg < ar, from_diag = jg == ar;
+      const int lim = is_q ? r + 1 : r;   // diagonal block: j < lim
       float out[16];
 #pragma unroll
       for (int jj = 0; jj < 16; ++jj) {
-        const int j = jg * 16 + jj;
-        float val = 0.f;
-        if (jg < ar)
-          val = ar == 1 ? vv[16 + jj] : (ar == 2 ? vv[32 + jj] : vv[48 + jj]);
-        else if (jg == ar)
-          val = (is_q ? (j <= r) : (j < r)) ? vv[jj] : 0.f;
-        out[jj] = val;
+        const float rv = ar == 1 ? vv[16 + jj] : (ar == 2 ? vv[32 + jj] : vv[48 + jj]);
+        const float dv_ = (from_diag && jg * 16 + jj < lim) ? vv[jj] : 0.f;
+        out[jj] = from_r ? rv : dv_;
       }
       if (!is_q) {
         const float br = s_beta[r];
@@ -638,8 +639,10 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
 #pragma unroll
       for (int e = 0; e < 8; e += 2) {
         const int j = j0 + e;
-        const float x0 = j <= r ? X[r * kLd + j] * s_beta[j] : 0.f;
-        const float x1 = j + 1 <= r ? X[r * kLd + j + 1] * s_beta[j + 1] : 0.f;
+        const float2 xv = *reinterpret_cast<const float2*>(X + r * kLd + j);
+        const float2 bv = *reinterpret_cast<const float2*>(s_beta + j);
+        const float x0 = j <= r ? xv.x * bv.x : 0.f;
+        const float x1 = j + 1 <= r ? xv.y * bv.y : 0.f;
         w[e >> 1] = pack_bf16x2(x0, x1);
       }
       *reinterpret_cast<uint4*>(smem + OFF_TM + tc::sw128<2>(r, j0, 64)) =
