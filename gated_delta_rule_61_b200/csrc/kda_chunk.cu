@@ -81,10 +81,10 @@ constexpr uint32_t OFF_XMAT = OFF_BG + 17408;  // X, fp32 [64][68]
 constexpr uint32_t OFF_ZBUF = OFF_BG + 34816;  // block products, fp32 [32][34]
 constexpr uint32_t OFF_NW = OFF_BG;            // after the solve: -W^T bf16 MN-major [c][r]
 constexpr uint32_t OFF_MISC = 188416;
-constexpr uint32_t MISC_GAMMA = 0, MISC_BETA = 512, MISC_GLAST = 768, MISC_PAIR = 1280,
+constexpr uint32_t MISC_GAMMA = 0, MISC_BETA = 512, MISC_PAIR = 1280,
                    MISC_GF = 17664, MISC_GL = 19712, MISC_MBAR = 21760, MISC_FULL = 21776,
-                   MISC_TMEM = 21784;
-constexpr uint32_t kSmemBytes = OFF_MISC + 21792 + 1024;
+                   MISC_TMEM = 21784, MISC_TOT4 = 21792;
+constexpr uint32_t kSmemBytes = OFF_MISC + 23840 + 1024;
 // State hand-over between the CTAs of a chain's cluster goes through the
 // chain's final_state slot in global memory (64 KiB, L2-resident): it is
 // written and read strictly in turn (CTA r writes S_n+1 after reading S_n;
@@ -368,7 +368,7 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
   // (the per-sub-chunk work of the off-diagonal Gram factors is balanced).
   const int pr = tid & 63, rg = tid >> 6, c0 = 2 * pr;
   float* s_pair = reinterpret_cast<float*>(smem + OFF_MISC + MISC_PAIR);   // [32][128]
-  float* s_glast = reinterpret_cast<float*>(smem + OFF_MISC + MISC_GLAST);
+  float* s_tot4 = reinterpret_cast<float*>(smem + OFF_MISC + MISC_TOT4);   // [4][128]
   // Inputs of the chunk about to be processed, loaded one chunk ahead.
   float2 lr[8];
   uint32_t kr[8], qr[8], vr[8];
@@ -419,22 +419,32 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         for (int i = 0; i < 8; ++i) s_beta[16 * (i >> 1) + 2 * rg + (i & 1)] = bt[i];
       }
       __syncthreads();
-      if (tid < 128) {
+      {
+        // Exclusive scan over rg within each sub-chunk (thread = (a, channel)),
+        // sub-chunk totals to s_tot4.
+        const int a = tid >> 7, c = tid & 127;
         float run = 0.f;
-#pragma unroll 8
-        for (int idx = 0; idx < 32; ++idx) {
-          const float x = s_pair[idx * 128 + tid];
-          s_pair[idx * 128 + tid] = run;
+#pragma unroll
+        for (int r8 = 0; r8 < 8; ++r8) {
+          const float x = s_pair[(a * 8 + r8) * 128 + c];
+          s_pair[(a * 8 + r8) * 128 + c] = run;
           run += x;
         }
-        s_glast[tid] = run;
-        s_gamma[tid] = __expf(run);
+        s_tot4[a * 128 + c] = run;
       }
       __syncthreads();
       flush_signal();
+      float tb0[4], tb1[4];   // totals of the sub-chunks before a
+      tb0[0] = tb1[0] = 0.f;
+#pragma unroll
+      for (int a = 1; a < 4; ++a) {
+        tb0[a] = tb0[a - 1] + s_tot4[(a - 1) * 128 + c0];
+        tb1[a] = tb1[a - 1] + s_tot4[(a - 1) * 128 + c0 + 1];
+      }
 #pragma unroll
       for (int a = 0; a < 4; ++a) {
-        const float b0 = s_pair[(a * 8 + rg) * 128 + c0], b1 = s_pair[(a * 8 + rg) * 128 + c0 + 1];
+        const float b0 = tb0[a] + s_pair[(a * 8 + rg) * 128 + c0];
+        const float b1 = tb1[a] + s_pair[(a * 8 + rg) * 128 + c0 + 1];
         g0[2 * a] = b0 + l0[2 * a];
         g0[2 * a + 1] = g0[2 * a] + l0[2 * a + 1];
         g1[2 * a] = b1 + l1[2 * a];
@@ -453,6 +463,8 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
           s_gl[a * 128 + c0] = g0[2 * a + 1];
           s_gl[a * 128 + c0 + 1] = g1[2 * a + 1];
         }
+        s_gamma[c0] = __expf(g0[7]);       // decay over the whole chunk
+        s_gamma[c0 + 1] = __expf(g1[7]);
       }
     }
     __syncthreads();
@@ -466,7 +478,7 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         mid0[a] = 0.5f * (s_gf[a * 128 + c0] + s_gl[a * 128 + c0]);
         mid1[a] = 0.5f * (s_gf[a * 128 + c0 + 1] + s_gl[a * 128 + c0 + 1]);
       }
-      const float gl0 = s_glast[c0], gl1 = s_glast[c0 + 1];
+      const float gl0 = s_gl[3 * 128 + c0], gl1 = s_gl[3 * 128 + c0 + 1];
       float dd0[4], dd1[4];   // dd[a] = e^{m_a - m_(a-1)}, a >= 1
       dd0[0] = dd1[0] = 1.f;
 #pragma unroll
