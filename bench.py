@@ -7,7 +7,10 @@ N(0, 0.1^2) fp32 initial state, chunk C=64 (inputs resident in HBM).
 Metric: tokens/s (positions B*T per second, all heads). The same JSON line
 carries the decode-step workload (B=256 sequences, H=32, d=128, fp32 state
 [256,32,128,128] updated in place, bf16 inputs, fresh inputs every step) as
-state-update GB/s, each with its roofline fraction.
+state-update GB/s, the packed variable-length prefill (64 sequences of
+log-uniform length in [128, 32768], H=32) and the long-context workload (one
+T=1,048,576 H=32 prefill, then 512 single-sequence decode steps replayed
+from a CUDA graph), each with its roofline fraction.
 
   python bench.py [--gpus N --steps K --warmup W]        # this library
   python bench.py --impl reference [...]                 # the fp64 CPU oracle
@@ -34,10 +37,13 @@ METRIC = "KDA prefill tokens/s & decode state GB/s (fraction of B200 roofline), 
 PREFILL = dict(B=4, T=8192, H=16, dk=128, dv=128, chunk=64, init_std=0.1)
 DECODE = dict(B=256, H=32, dk=128, dv=128, std=0.05)
 VARLEN = dict(H=32)
+LONG = dict(T=1 << 20, H=32, decode_steps=512)
 BYTES_PER_HEAD_TOKEN = 3 * 256 + 512 + 4 + 256        # q,k,v + log_alpha + beta + o
 FLOPS_PER_HEAD_TOKEN = 6 * 128 * 128 + 2 * 64 * (3 * 128 + 2 * 128)   # dense tiles, C = 64
 PROFILE = os.path.join(ROOT, "profiles", "chunk64_prefill_b4_t8192_h16.txt")
 KERNEL_SRC = os.path.join(ROOT, "gated_delta_rule_61_b200", "csrc", "kda_chunk.cu")
+DECODE_PROFILE = os.path.join(ROOT, "profiles", "decode_step_b256_h32.txt")
+DECODE_SRC = os.path.join(ROOT, "gated_delta_rule_61_b200", "csrc", "kda_decode.cu")
 
 
 def peaks():
@@ -49,12 +55,12 @@ def peaks():
         return 6650.0, 1590.0, "fallback"
 
 
-def kernel_traffic():
-    """dram bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel source (else None)."""
+def kernel_traffic(profile=PROFILE, src=KERNEL_SRC):
+    """dram bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
     try:
-        text = open(PROFILE).read()
-        src_hash = hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()[:16]
+        text = open(profile).read()
+        src_hash = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
         fields = dict(line.split(":", 1) for line in text.splitlines() if ":" in line)
         if fields.get("kernel_source_sha256_16", "").strip() != src_hash:
             return None
@@ -298,7 +304,8 @@ def bench_ours(args):
                "tokens_per_s": world * D["B"] / (dms * 1e-3),
                "workload": "KDA decode B=256 H=32 dk=dv=128, fp32 state in place, bf16 inputs",
                "roofline": {"bound": "hbm", "achieved": gbs / world, "peak": hbm,
-                            "unit": "GB/s", "frac": gbs / world / hbm, "traffic": None,
+                            "unit": "GB/s", "frac": gbs / world / hbm,
+                            "traffic": kernel_traffic(DECODE_PROFILE, DECODE_SRC),
                             "peak_kind": peak_kind}}
         del steps_in, S
     # ---------------- packed variable-length prefill ----------------
@@ -337,6 +344,72 @@ def bench_ours(args):
                             "frac": vgbs / hbm, "traffic": None, "peak_kind": peak_kind},
                "gpu_launches_per_step": 2}
         del vin, vo, vs
+    # ---------------- long context: one 1M-token prefill, then graph-replayed decode ----------------
+    lng = None
+    if not args.no_long:
+        L = LONG
+        lin = prefill_inputs(1, L["T"], L["H"], 128, 128, dtype=torch.bfloat16, seed=4000 + rank,
+                             device=dev)
+        lo = torch.empty_like(lin["v"])
+        ls = torch.empty(1, L["H"], 128, 128, dtype=torch.float32, device=dev)
+
+        def lstep():
+            kda.prefill(lin["q"], lin["k"], lin["v"], lin["log_alpha"], lin["beta"], chunk=64,
+                        o=lo, final_state=ls, stream=stream)
+
+        lstep()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_l = 3
+        a.record(stream)
+        for _ in range(n_l):
+            lstep()
+        b.record(stream)
+        barrier(world)
+        lms = max_over_ranks(a.elapsed_time(b), world) / n_l
+        lbytes = L["T"] * L["H"] * BYTES_PER_HEAD_TOKEN + L["H"] * 128 * 128 * 4
+        lgbs = lbytes / (lms * 1e-3) / 1e9
+        del lin, lo
+        # decode from the prefill's final state: B=1, so a step is a few microseconds
+        # and launch overhead matters; the steps are captured once in a CUDA graph
+        n_d = L["decode_steps"]
+        dins = [decode_inputs(1, L["H"], 128, 128, dtype=torch.bfloat16, seed=4000 + rank,
+                              step=i, device=dev) for i in range(n_d)]
+        dout = torch.empty(n_d, 1, L["H"], 128, dtype=torch.bfloat16, device=dev)
+        s_work = ls.clone()
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        with torch.cuda.graph(graph, stream=cap):
+            for i, d in enumerate(dins):
+                kda.decode_step(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], s_work,
+                                o=dout[i], stream=cap)
+        stream.wait_stream(cap)
+        for _ in range(args.warmup):
+            s_work.copy_(ls)
+            graph.replay()
+        barrier(world)
+        ev_d = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(n_l)]
+        for a, b in ev_d:
+            s_work.copy_(ls)       # every replay starts from the prefill's final state
+            a.record(stream)
+            graph.replay()
+            b.record(stream)
+        barrier(world)
+        gms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in ev_d), world)
+        dus = gms * 1e3 / n_d
+        dbytes = L["H"] * (2 * 128 * 128 * 4 + BYTES_PER_HEAD_TOKEN)
+        lng = {"value": world * L["T"] / (lms * 1e-3), "unit": "tokens/s", "ms_per_step": lms,
+               "workload": "KDA long-context prefill B=1 T=%d H=32 d=128 bf16, C=64, zero "
+                           "initial state; then %d decode steps (CUDA graph)" % (L["T"], n_d),
+               "roofline": {"bound": "hbm", "achieved": lgbs, "peak": hbm, "unit": "GB/s",
+                            "frac": lgbs / hbm, "traffic": None, "peak_kind": peak_kind},
+               "decode": {"us_per_step": dus, "steps": n_d, "unit": "GB/s",
+                          "value": dbytes / (dus * 1e-6) / 1e9,
+                          "frac": dbytes / (dus * 1e-6) / 1e9 / hbm}}
+        del graph, dins, dout, s_work, ls
+        torch.cuda.empty_cache()
     clk.__exit__(None, None, None)
 
     # ---------------- end to end through the public API (host buffers) ----------------
@@ -392,7 +465,7 @@ def bench_ours(args):
                          "peak_kind": peak_kind, "kernel_ms": kernel_ms,
                          "tensor": {"achieved_tflops": tflops, "peak_tflops": bf16_tf,
                                     "frac": tflops / bf16_tf}},
-            "decode": dec, "varlen": var, "e2e": e2e, "cpu_baseline": cpu,
+            "decode": dec, "varlen": var, "long": lng, "e2e": e2e, "cpu_baseline": cpu,
             "gpu_launches": args.steps, "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
@@ -411,6 +484,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-varlen", action="store_true")
+    ap.add_argument("--no-long", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--ref-budget", type=float, default=8.0)

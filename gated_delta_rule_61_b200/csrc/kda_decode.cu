@@ -10,55 +10,50 @@
 // pass over S, so the state is read once and written once: the kernel is
 // bound by HBM bandwidth (about 2 * dk * dv * 4 bytes per head).
 //
-// Layout: one CTA per (sequence, head); 256 threads = 8 warps. Lane l owns
-// value columns [VPL*l, VPL*l + VPL) (VPL = dv / 32, one 128-bit or 64-bit
-// vector); warp w owns key rows w, w + 8, ... (dk / 8 rows). A warp therefore
-// reads whole contiguous rows of S (coalesced 512-byte rows for dv = 128).
+// Layout: SPLIT CTAs per (sequence, head), each owning a slice of the value
+// columns; 256 threads = 8 warps; every lane streams 128-bit vectors of whole
+// contiguous rows, holds its rows in registers between the read and the
+// write, and the two column reductions go through shuffles and one small
+// shared-memory exchange.
 #include "kda_common.cuh"
 
 namespace kda {
 
-template <int N> struct VecF;
-template <> struct VecF<4> {
-  using T = float4;
-  static __device__ __forceinline__ void unpack(const T& v, float* e) {
-    e[0] = v.x; e[1] = v.y; e[2] = v.z; e[3] = v.w;
-  }
-  static __device__ __forceinline__ T pack(const float* e) { return make_float4(e[0], e[1], e[2], e[3]); }
-};
-template <> struct VecF<2> {
-  using T = float2;
-  static __device__ __forceinline__ void unpack(const T& v, float* e) { e[0] = v.x; e[1] = v.y; }
-  static __device__ __forceinline__ T pack(const float* e) { return make_float2(e[0], e[1]); }
-};
-
-template <typename TIn, int DK, int DV>
-__global__ void __launch_bounds__(256, 2)
+// SPLIT CTAs share a head: CTA (head, slice) owns value columns
+// [slice * DV / SPLIT, +DV / SPLIT) (value columns evolve independently given
+// k, alpha, beta and their v entries). Within a CTA each lane owns one 4-column
+// group; LPR = columns / 4 lanes cover a row, so a warp instruction reads RPI =
+// 32 / LPR whole rows (512 contiguous bytes per warp for 128 columns).
+template <typename TIn, int DK, int DV, int SPLIT>
+__global__ void __launch_bounds__(256, 2 * SPLIT)
 decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                    const TIn* __restrict__ v, const float* __restrict__ log_alpha,
                    const float* __restrict__ beta, float* __restrict__ state,
                    TIn* __restrict__ o) {
   constexpr int kWarps = 8;
-  constexpr int VPL = DV / 32;          // value columns per lane
-  constexpr int RPW = DK / kWarps;      // key rows per warp
-  using V = VecF<VPL>;
-  using VT = typename V::T;
+  constexpr int CW = DV / SPLIT;          // value columns of this CTA
+  constexpr int LPR = CW / 4;             // lanes per row (one float4 each)
+  constexpr int RPI = 32 / LPR;           // rows per warp instruction
+  constexpr int NI = DK / (kWarps * RPI); // float4 per thread
+  static_assert(CW % 4 == 0 && 32 % LPR == 0 && DK % (kWarps * RPI) == 0, "shape");
 
-  const int head = blockIdx.x;          // flat (b, h)
+  const int head = blockIdx.x / SPLIT, slice = blockIdx.x % SPLIT;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cg = lane % LPR, sub = lane / LPR;
+  const int col = slice * CW + 4 * cg;
 
   __shared__ float s_k[DK], s_q[DK], s_a[DK];
-  __shared__ float s_red[kWarps][2][DV];
+  __shared__ float4 s_red[kWarps][2][LPR];
   __shared__ float s_kq[kWarps];
 
   float* S = state + (size_t)head * DK * DV;
 
   // Issue the state loads first: they are the bytes that matter.
-  float s[RPW][VPL];
+  float4 s[NI];
 #pragma unroll
-  for (int i = 0; i < RPW; ++i) {
-    const int row = warp + i * kWarps;
-    V::unpack(__ldcs(reinterpret_cast<const VT*>(S + (size_t)row * DV) + lane), s[i]);
+  for (int i = 0; i < NI; ++i) {
+    const int row = (warp + i * kWarps) * RPI + sub;
+    s[i] = __ldcs(reinterpret_cast<const float4*>(S + (size_t)row * DV + col));
   }
 
   // Small per-head vectors: k, q, alpha = exp(log_alpha); k . q per warp.
@@ -77,53 +72,59 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
   __syncthreads();
 
   // Decay rows and accumulate partial r = S'^T k and p = S'^T q.
-  float r[VPL], p[VPL];
+  float4 r = make_float4(0.f, 0.f, 0.f, 0.f), p = r;
 #pragma unroll
-  for (int j = 0; j < VPL; ++j) r[j] = p[j] = 0.f;
-#pragma unroll
-  for (int i = 0; i < RPW; ++i) {
-    const int row = warp + i * kWarps;
+  for (int i = 0; i < NI; ++i) {
+    const int row = (warp + i * kWarps) * RPI + sub;
     const float a = s_a[row], kk = s_k[row], qq = s_q[row];
-#pragma unroll
-    for (int j = 0; j < VPL; ++j) {
-      s[i][j] *= a;
-      r[j] = fmaf(s[i][j], kk, r[j]);
-      p[j] = fmaf(s[i][j], qq, p[j]);
-    }
+    s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
+    r.x = fmaf(s[i].x, kk, r.x); r.y = fmaf(s[i].y, kk, r.y);
+    r.z = fmaf(s[i].z, kk, r.z); r.w = fmaf(s[i].w, kk, r.w);
+    p.x = fmaf(s[i].x, qq, p.x); p.y = fmaf(s[i].y, qq, p.y);
+    p.z = fmaf(s[i].z, qq, p.z); p.w = fmaf(s[i].w, qq, p.w);
   }
 #pragma unroll
-  for (int j = 0; j < VPL; ++j) {
-    s_red[warp][0][lane * VPL + j] = r[j];
-    s_red[warp][1][lane * VPL + j] = p[j];
+  for (int off = LPR; off < 32; off <<= 1) {   // lanes holding the same columns
+    r.x += __shfl_xor_sync(0xffffffffu, r.x, off); r.y += __shfl_xor_sync(0xffffffffu, r.y, off);
+    r.z += __shfl_xor_sync(0xffffffffu, r.z, off); r.w += __shfl_xor_sync(0xffffffffu, r.w, off);
+    p.x += __shfl_xor_sync(0xffffffffu, p.x, off); p.y += __shfl_xor_sync(0xffffffffu, p.y, off);
+    p.z += __shfl_xor_sync(0xffffffffu, p.z, off); p.w += __shfl_xor_sync(0xffffffffu, p.w, off);
+  }
+  if (sub == 0) {
+    s_red[warp][0][cg] = r;
+    s_red[warp][1][cg] = p;
   }
   __syncthreads();
 
   float kq = 0.f;
 #pragma unroll
   for (int w = 0; w < kWarps; ++w) kq += s_kq[w];
-  const float b = __ldg(beta + head);
-  float d[VPL];
+  r = make_float4(0.f, 0.f, 0.f, 0.f);
+  p = r;
 #pragma unroll
-  for (int j = 0; j < VPL; ++j) {
-    float rr = 0.f, pp = 0.f;
+  for (int w = 0; w < kWarps; ++w) {
+    const float4 a = s_red[w][0][cg], b = s_red[w][1][cg];
+    r.x += a.x; r.y += a.y; r.z += a.z; r.w += a.w;
+    p.x += b.x; p.y += b.y; p.z += b.z; p.w += b.w;
+  }
+  const float bb = __ldg(beta + head);
+  const float rr[4] = {r.x, r.y, r.z, r.w}, pp[4] = {p.x, p.y, p.z, p.w};
+  float d[4];
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      rr += s_red[w][0][lane * VPL + j];
-      pp += s_red[w][1][lane * VPL + j];
-    }
-    const int col = lane * VPL + j;
-    d[j] = b * (Io<TIn>::load(v + (size_t)head * DV + col) - rr);
-    if (warp == 0) Io<TIn>::store(o + (size_t)head * DV + col, fmaf(kq, d[j], pp));
+  for (int j = 0; j < 4; ++j) {
+    d[j] = bb * (Io<TIn>::load(v + (size_t)head * DV + col + j) - rr[j]);
+    if (warp == 0 && sub == 0)
+      Io<TIn>::store(o + (size_t)head * DV + col + j, fmaf(kq, d[j], pp[j]));
   }
 
   // S = S' + k d^T, written once.
 #pragma unroll
-  for (int i = 0; i < RPW; ++i) {
-    const int row = warp + i * kWarps;
+  for (int i = 0; i < NI; ++i) {
+    const int row = (warp + i * kWarps) * RPI + sub;
     const float kk = s_k[row];
-#pragma unroll
-    for (int j = 0; j < VPL; ++j) s[i][j] = fmaf(kk, d[j], s[i][j]);
-    __stcs(reinterpret_cast<VT*>(S + (size_t)row * DV) + lane, V::pack(s[i]));
+    s[i].x = fmaf(kk, d[0], s[i].x); s[i].y = fmaf(kk, d[1], s[i].y);
+    s[i].z = fmaf(kk, d[2], s[i].z); s[i].w = fmaf(kk, d[3], s[i].w);
+    __stcs(reinterpret_cast<float4*>(S + (size_t)row * DV + col), s[i]);
   }
 }
 
@@ -131,7 +132,8 @@ template <typename TIn, int DK, int DV>
 static cudaError_t launch_decode_t(const void* q, const void* k, const void* v,
                                    const float* la, const float* beta, float* state,
                                    void* o, int n_heads, cudaStream_t stream) {
-  decode_step_kernel<TIn, DK, DV><<<n_heads, 256, 0, stream>>>(
+  constexpr int kSplit = DV == 128 ? 2 : 1;
+  decode_step_kernel<TIn, DK, DV, kSplit><<<n_heads * kSplit, 256, 0, stream>>>(
       (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, state, (TIn*)o);
   return cudaGetLastError();
 }

@@ -245,6 +245,40 @@ def test_decode_steps(dtype, dk, dv):
         assert_close(S_gpu, S_ref, TOL_F32, "decode state step %d" % step)
 
 
+def test_decode_graph_replay_matches_eager_and_oracle():
+    """Decode steps captured once in a CUDA graph (how a single-sequence decode
+    loop amortises launch latency) give the same bits as eager launches, and
+    the oracle's values."""
+    B, H, d, n = 1, 32, 128, 6
+    S0 = decode_state(B, H, d, d, std=0.05, seed=21)
+    ins = [_to(decode_inputs(B, H, d, d, dtype=torch.bfloat16, seed=21, step=i))
+           for i in range(n)]
+    names = ("q", "k", "v", "log_alpha", "beta")
+    S_eager = S0.to(DEV)
+    o_eager = [kda.decode_step(*(g[x] for x in names), S_eager) for g in ins]
+    S_graph = S0.to(DEV)
+    o_graph = torch.empty(n, B, H, d, dtype=torch.bfloat16, device=DEV)
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(graph, stream=cap):
+        for i, g in enumerate(ins):
+            kda.decode_step(*(g[x] for x in names), S_graph, o=o_graph[i], stream=cap)
+    torch.cuda.current_stream().wait_stream(cap)
+    S_graph.copy_(S0.to(DEV))     # capture does not run the kernels; start from S0
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(S_graph, S_eager)
+    for i in range(n):
+        assert torch.equal(o_graph[i], o_eager[i])
+    S_ref = S0.double().numpy()
+    for i in range(n):
+        o_ref, S_ref = oracle.kda_decode_step(*(ins[i][x].cpu() for x in names), S_ref)
+        assert_close(o_graph[i], o_ref, TOL_BF16_O, "graph decode o step %d" % i)
+    assert_close(S_graph, S_ref, TOL_F32, "graph decode state")
+    del graph
+
+
 def test_prefill_then_decode_equals_longer_prefill():
     inp = _to(prefill_inputs(2, 129, 2, 128, 128, dtype=torch.bfloat16, seed=15, init_std=0.1))
     o_all, s_all = kda.prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
