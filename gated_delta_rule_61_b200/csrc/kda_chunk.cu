@@ -328,18 +328,6 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
   const uint32_t tmem = *tmem_slot;
   uint32_t phase = 0, full_phase = 0;
   bool ok = true;
-  bool signal_pending = false;   // a state hand-over written but not yet announced
-  // Announce a written hand-over to the next CTA of the ring (thread 0, after
-  // a CTA barrier that follows every thread's stores).
-  auto flush_signal = [&]() {
-    if (kPair && signal_pending) {
-      if (tid == 0) {
-        asm volatile("fence.acq_rel.cluster;" ::: "memory");
-        tc::mbar_remote_arrive(tc::mapa_shared(mbar_full, (uint32_t)((rank + 1) % kRing)));
-      }
-      signal_pending = false;
-    }
-  };
 
   const int quad = warp & 3, grp = warp >> 2;
   const int m = quad * 32 + lane;
@@ -394,14 +382,14 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     const long long tf = t_begin + (long long)rank * C;
     load_rows(tf, (int)((t_end - tf) < C ? (t_end - tf) : C));
   }
-
-  for (int n = rank; n < n_chunks; n += step) {
-    const long long t0 = t_begin + (long long)n * C;
-
-    // ---- P1: cumulative gates and operand tiles --------------------------
-    // Cumulative sums: pair sums per (sub-chunk, rg) -> one exclusive scan
-    // over the 32 pairs per channel -> each thread adds its own rows.
-    float g0[8], g1[8];
+  // Cumulative gates of a chunk from the prefetched log_alpha rows (lr):
+  // pair sums per (sub-chunk, rg) -> one exclusive scan over the 32 pairs per
+  // channel -> each thread adds its own rows. Writes g0/g1 (registers), beta,
+  // the first and last g of every sub-chunk and the chunk's decay e^{g_last}
+  // to shared memory. Runs for the next chunk while the current chunk's
+  // D/O MMA is in flight; it touches no operand tile.
+  float g0[8], g1[8];
+  auto gates = [&]() {
     {
       float l0[8], l1[8];
 #pragma unroll
@@ -433,7 +421,6 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         s_tot4[a * 128 + c] = run;
       }
       __syncthreads();
-      flush_signal();
       float tb0[4], tb1[4];   // totals of the sub-chunks before a
       tb0[0] = tb1[0] = 0.f;
 #pragma unroll
@@ -468,6 +455,16 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       }
     }
     __syncthreads();
+  };
+  if (rank < n_chunks) gates();
+
+  for (int n = rank; n < n_chunks; n += step) {
+    const long long t0 = t_begin + (long long)n * C;
+
+    // ---- P1: operand tiles. The gates were formed during the previous own
+    // chunk's D/O MMA, except with four CTAs per chain, where that MMA is on
+    // the chain's critical path and the gates are formed here. -----------
+    if (kRing > 2 && n != rank) gates();
     {
       // Sub-chunk midpoints m_a and the per-channel factors, from five
       // exponentials per channel: e^{m_0}, e^{m_a - m_(a-1)} and e^{g_last - m_3};
@@ -594,29 +591,42 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     if (!ok) break;
 
     // ---- P3: rows of M_kk (lanes 0..63) and M_qk (lanes 64..127) ---------
-    // Warp (quad, grp) assembles columns j in [16 grp, 16 grp + 16).
+    // Warp (quad, grp) assembles columns j in [16 grp, 16 grp + 16) for its 32
+    // rows, which fall in two sub-chunks: a_lo (lanes 0-15) and a_lo + 1.
+    // Column block jg of a row in sub-chunk a comes from the R_a set (jg < a),
+    // from the diagonal set under the causal mask (jg == a), or is zero, so a
+    // warp needs at most two 16-column loads, chosen warp-uniformly.
     {
       const int row = m;
       const bool is_q = row >= 64;
-      const int r = row & 63, ar = r >> 4;
-      const int jg = grp;
+      const int r = row & 63;
+      const int jg = grp, a_lo = 2 * (quad & 1), a_hi = a_lo + 1;
+      const bool hi = lane >= 16;
       const uint32_t tb = tmem + lane_off + TM_G;
-      // diag block columns, then the R sets that cover columns of group jg.
-      const uint32_t c_r1 = 64 + 16 * jg, c_r2 = 80 + 16 * jg, c_r3 = 112 + 16 * jg;
-      float vv[64];
-      tc::tmem_ld16x4(tb + 16 * jg, tb + (jg == 0 ? c_r1 : 16 * jg),
-                      tb + (jg <= 1 ? c_r2 : 16 * jg), tb + (jg <= 2 ? c_r3 : 16 * jg), vv);
-      // Branch-free selection (the row's sub-chunk ar differs between lanes):
-      // column block jg < ar comes from R_ar, jg == ar from the diagonal set
-      // under the causal mask, jg > ar is zero.
-      const bool from_r = jg < ar, from_diag = jg == ar;
-      const int lim = is_q ? r + 1 : r;   // diagonal block: j < lim
+      auto r_col = [&](int a) { return (uint32_t)((a == 1 ? 64 : a == 2 ? 80 : 112) + 16 * jg); };
+      float vv[32];
+      if (jg < a_lo) {
+        tc::tmem_ld16x2(tb + r_col(a_lo), tb + r_col(a_hi), vv);
+      } else if (jg == a_lo) {
+        tc::tmem_ld16x2(tb + 16 * jg, tb + r_col(a_hi), vv);
+      } else if (jg == a_hi) {
+        tc::tmem_ld16x2(tb + 16 * jg, tb + 16 * jg, vv);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) vv[i] = 0.f;
+      }
+      // vv[0..15]: block for the a_lo rows (or the diagonal set), vv[16..31]:
+      // block for the a_hi rows. Diagonal entries keep j < r (k rows) or
+      // j <= r (q rows).
+      const int lim = is_q ? r + 1 : r;
+      const bool lo_diag = jg == a_lo, hi_diag = jg == a_hi;
       float out[16];
 #pragma unroll
       for (int jj = 0; jj < 16; ++jj) {
-        const float rv = ar == 1 ? vv[16 + jj] : (ar == 2 ? vv[32 + jj] : vv[48 + jj]);
-        const float dv_ = (from_diag && jg * 16 + jj < lim) ? vv[jj] : 0.f;
-        out[jj] = from_r ? rv : dv_;
+        const bool causal = jg * 16 + jj < lim;
+        const float lo = lo_diag ? (causal ? vv[jj] : 0.f) : (jg < a_lo ? vv[jj] : 0.f);
+        const float hv = hi_diag ? (causal ? vv[jj] : 0.f) : (jg < a_hi ? vv[16 + jj] : 0.f);
+        out[jj] = hi ? hv : lo;
       }
       if (!is_q) {
         const float br = s_beta[r];
@@ -772,6 +782,7 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       }
       tc::mma_commit(mbar);
     }
+    if (kRing <= 2 && n + step < n_chunks) gates();   // next own chunk, while the MMAs run
     ok = cta_wait(mbar, phase, 3);
     phase ^= 1;
     if (!ok) break;
@@ -805,21 +816,18 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       for (int v4 = 0; v4 < 8; ++v4)
         __stcg(slot + xfer_chunk(m, grp * 8 + v4),
                make_float4(s[4 * v4], s[4 * v4 + 1], s[4 * v4 + 2], s[4 * v4 + 3]));
-      // With two CTAs per chain the partner is still busy with its own chunk
-      // preparation, so it is told later (signal_pending: after a CTA barrier
-      // in the next chunk, once the stores have landed and the release fence
-      // is cheap). With four, the hand-over is on the critical path: tell it
-      // now.
-      signal_pending = true;
-      if (kRing > 2) {
-        __syncthreads();
-        flush_signal();
+      // Announce it: thread 0, after a CTA barrier that follows every
+      // thread's stores, releases them at cluster scope and arrives on the
+      // next CTA's barrier.
+      __syncthreads();
+      if (tid == 0) {
+        asm volatile("fence.acq_rel.cluster;" ::: "memory");
+        tc::mbar_remote_arrive(tc::mapa_shared(mbar_full, (uint32_t)((rank + 1) % kRing)));
       }
     }
   }
 
   __syncthreads();
-  flush_signal();
   if (ok && n_chunks > rank) {
     const int n_mine = rank + step * ((n_chunks - 1 - rank) / step);   // this CTA's last chunk
     const long long t_last = t_begin + (long long)n_mine * C;
