@@ -570,8 +570,15 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       }
       tc::mma_commit(mbar);
     }
-    if (n + step < n_chunks) {  // warm L2 with this CTA's next chunk
+    // While the Gram MMA runs: load this CTA's next chunk into registers (its
+    // inputs are consumed by then: the gates in the D/O MMA wait, the tiles
+    // in P1) and warm L2 with the chunk after it.
+    if (n + step < n_chunks) {
       const long long t1 = t0 + (long long)step * C;
+      load_rows(t1, (int)((t_end - t1) < C ? (t_end - t1) : C));
+    }
+    if (n + 2 * step < n_chunks) {
+      const long long t1 = t0 + (long long)(2 * step) * C;
       const int row = tid >> 3, part = tid & 7;
       if (t1 + row < t_end) {
         const size_t tok = (size_t)(t1 + row) * H + head;
@@ -707,12 +714,6 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       tc::tmem_st16(tb + 16, s + 16);
       tc::tmem_wait_st();
     }
-    // This chunk's inputs are consumed: load the next chunk's now, so the
-    // loads are in flight during the state MMAs.
-    if (n + step < n_chunks) {
-      const long long t1 = t0 + (long long)step * C;
-      load_rows(t1, (int)((t_end - t1) < C ? (t_end - t1) : C));
-    }
     ok = cta_wait(mbar, phase, 2);
     phase ^= 1;
     if (!ok) break;
@@ -816,14 +817,13 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       for (int v4 = 0; v4 < 8; ++v4)
         __stcg(slot + xfer_chunk(m, grp * 8 + v4),
                make_float4(s[4 * v4], s[4 * v4 + 1], s[4 * v4 + 2], s[4 * v4 + 3]));
-      // Announce it: thread 0, after a CTA barrier that follows every
-      // thread's stores, releases them at cluster scope and arrives on the
-      // next CTA's barrier.
+      // Announce it: after a CTA barrier that orders every thread's stores
+      // before it, thread 0 arrives on the next CTA's barrier with release
+      // semantics at cluster scope (cumulative over the stores the barrier
+      // ordered); the receiver's acquire wait pairs with it.
       __syncthreads();
-      if (tid == 0) {
-        asm volatile("fence.acq_rel.cluster;" ::: "memory");
+      if (tid == 0)
         tc::mbar_remote_arrive(tc::mapa_shared(mbar_full, (uint32_t)((rank + 1) % kRing)));
-      }
     }
   }
 
