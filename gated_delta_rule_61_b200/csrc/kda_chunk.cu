@@ -152,9 +152,10 @@ __device__ __forceinline__ void cta_sync_tc() {
 // X = (I + N)^-1 for the strictly lower 64 x 64 matrix N (row stride kLd),
 // as a recursive 2 x 2 block inverse: for a unit lower block matrix
 // [[A, 0], [C, D]] the inverse is [[A^-1, 0], [-D^-1 C A^-1, D^-1]].
-// Level 1 inverts the four 16 x 16 diagonal blocks by forward substitution,
-// level 2 fills the two 16 x 16 blocks below them, level 3 the 32 x 32 block.
-// Entries above the diagonal are never read.
+// Level 1 inverts the four 16 x 16 diagonal blocks by forward substitution
+// (their entries above the diagonal come out as exact zeros), level 2 fills
+// the two 16 x 16 blocks below them, level 3 the 32 x 32 block. Entries above
+// the diagonal outside the diagonal blocks are never read.
 __device__ __forceinline__ void invert_diag_block(const float* N, float* X, int t) {
   const int base = (t >> 4) * 16, col = t & 15;
   float x[16];
@@ -175,29 +176,57 @@ __device__ __forceinline__ void invert_diag_block(const float* N, float* X, int 
 }
 
 __device__ __forceinline__ void invert_unit_lower64(const float* N, float* X, float* Z, int t) {
-  if (t < 64) invert_diag_block(N, X, t);
-  __syncthreads();
-  // Level 2: blocks (1,0) and (3,2): Z_p = N_{b a} X_{a a}, X_{b a} = -X_{b b} Z_p.
-  {
-    const int p = t >> 8, rr = (t >> 4) & 15, cc = t & 15;
-    const int a = 2 * p * 16, b = a + 16;
-    float z0 = 0.f, z1 = 0.f;
+  // Levels 1 and 2 in warps 0 and 1: warp p inverts the diagonal blocks 2p
+  // and 2p + 1, then fills block (2p + 1, 2p) below them with two 16 x 16 x 16
+  // tf32 m16n8k8 products (tf32 rounding there is below the bf16 rounding T
+  // receives next), so nothing outside the warp is waited for until level 3.
+  if (t < 64) {
+    invert_diag_block(N, X, t);
+    __syncwarp();
+    const int p = t >> 5, lane = t & 31, gid = lane >> 2, tig = lane & 3;
+    const int a = 32 * p, b = a + 16;
+    float* Zp = Z + p * 16 * 34;
+    // Z_p = N_{b a} X_{a a}  (X_{a a} lower triangular; its upper entries are zeros)
 #pragma unroll
-    for (int kk = 0; kk < 16; kk += 2) {
-      z0 += N[(b + rr) * kLd + a + kk] * X[(a + kk) * kLd + a + cc];
-      z1 += N[(b + rr) * kLd + a + kk + 1] * X[(a + kk + 1) * kLd + a + cc];
-    }
-    Z[(p * 16 + rr) * 34 + cc] = z0 + z1;
-    __syncthreads();
-    float x0 = 0.f, x1 = 0.f;
+    for (int nt = 0; nt < 2; ++nt) {
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int kk = 0; kk < 16; kk += 2) {
-      x0 += X[(b + rr) * kLd + b + kk] * Z[(p * 16 + kk) * 34 + cc];
-      x1 += X[(b + rr) * kLd + b + kk + 1] * Z[(p * 16 + kk + 1) * 34 + cc];
+      for (int kt = 0; kt < 2; ++kt) {
+        if (kt < nt) continue;   // rows k < 8 nt of X_{a a} vanish in these columns
+        const int k0 = 8 * kt + tig, c = 8 * nt + gid;
+        const uint32_t av[4] = {to_tf32(N[(b + gid) * kLd + a + k0]),
+                                to_tf32(N[(b + gid + 8) * kLd + a + k0]),
+                                to_tf32(N[(b + gid) * kLd + a + k0 + 4]),
+                                to_tf32(N[(b + gid + 8) * kLd + a + k0 + 4])};
+        const uint32_t bv[2] = {to_tf32(X[(a + k0) * kLd + a + c]),
+                                to_tf32(X[(a + k0 + 4) * kLd + a + c])};
+        mma_16x8x8_tf32(d, av, bv);
+      }
+      const int zc = 8 * nt + 2 * tig;
+      *reinterpret_cast<float2*>(Zp + gid * 34 + zc) = make_float2(d[0], d[1]);
+      *reinterpret_cast<float2*>(Zp + (gid + 8) * 34 + zc) = make_float2(d[2], d[3]);
     }
-    X[(b + rr) * kLd + a + cc] = -(x0 + x1);
-    __syncthreads();
+    __syncwarp();
+    // X_{b a} = -X_{b b} Z_p
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int kt = 0; kt < 2; ++kt) {
+        const int k0 = 8 * kt + tig, c = 8 * nt + gid;
+        const uint32_t av[4] = {to_tf32(X[(b + gid) * kLd + b + k0]),
+                                to_tf32(X[(b + gid + 8) * kLd + b + k0]),
+                                to_tf32(X[(b + gid) * kLd + b + k0 + 4]),
+                                to_tf32(X[(b + gid + 8) * kLd + b + k0 + 4])};
+        const uint32_t bv[2] = {to_tf32(Zp[k0 * 34 + c]), to_tf32(Zp[(k0 + 4) * 34 + c])};
+        mma_16x8x8_tf32(d, av, bv);
+      }
+      const int xc = a + 8 * nt + 2 * tig;
+      *reinterpret_cast<float2*>(X + (b + gid) * kLd + xc) = make_float2(-d[0], -d[1]);
+      *reinterpret_cast<float2*>(X + (b + gid + 8) * kLd + xc) = make_float2(-d[2], -d[3]);
+    }
   }
+  __syncthreads();
   // Level 3: Z = N[32:64, 0:32] X[0:32, 0:32];  X[32:64, 0:32] = -X[32:64, 32:64] Z,
   // as tf32 m16n8k8 MMAs: warps 0..7 each own one 16 x 8 tile of the 32 x 32 result.
   const int warp = t >> 5, lane = t & 31, gid = lane >> 2, tig = lane & 3;
@@ -218,8 +247,15 @@ __device__ __forceinline__ void invert_unit_lower64(const float* N, float* X, fl
     const int zr = 16 * mt + gid, zc = 8 * nt + 2 * tig;
     *reinterpret_cast<float2*>(Z + zr * 34 + zc) = make_float2(d[0], d[1]);
     *reinterpret_cast<float2*>(Z + (zr + 8) * 34 + zc) = make_float2(d[2], d[3]);
+    // The upper result tile (mt = 0) needs only this warp's own Z tile; the
+    // lower one (mt = 1) also needs its partner's (warp nt), which announces
+    // it on named barrier 4 + nt without waiting.
+    if (mt == 0)
+      asm volatile("bar.arrive %0, 64;" ::"r"(4 + nt) : "memory");
+    else
+      asm volatile("bar.sync %0, 64;" ::"r"(4 + nt) : "memory");
+    __syncwarp();
   }
-  __syncthreads();
   if (warp < 8) {
     float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
