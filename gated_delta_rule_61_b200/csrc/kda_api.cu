@@ -19,6 +19,15 @@ cudaError_t launch_chunk64(const void* q, const void* k, const void* v, const fl
 
 static bool head_size_ok(int d) { return d == 64 || d == 128; }
 
+// The chunked kernel moves q, k, v, o, log_alpha and the state hand-over in
+// 8- and 16-byte vectors.
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+bool chunk_pointers_aligned(const void* q, const void* k, const void* v, const float* la,
+                            const void* o, const float* sT) {
+  return aligned16(q) && aligned16(k) && aligned16(v) && aligned16(la) && aligned16(o) &&
+         (!sT || aligned16(sT));
+}
+
 }  // namespace kda
 
 extern "C" {
@@ -70,6 +79,8 @@ kda_status kda_prefill(const void* q, const void* k, const void* v, const float*
   cudaError_t err;
   if (use_chunk) {
     if (dk != 128 || dv != 128) return KDA_ERR_UNSUPPORTED;
+    if (tokens > 0 && !kda::chunk_pointers_aligned(q, k, v, log_alpha, o, final_state))
+      return KDA_ERR_INVALID_ARG;
     const size_t need = kda_prefill_workspace_bytes(n_seq, cu_seqlens != nullptr);
     if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
     if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255)) return KDA_ERR_WORKSPACE;

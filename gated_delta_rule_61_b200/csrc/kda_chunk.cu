@@ -104,15 +104,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&p);
 }
 
-// 1/x for normal positive x by Newton-Raphson on the reciprocal (two steps
-// from an initial estimate read off the IEEE-754 exponent and mantissa bits,
-// the classic "magic constant" start): relative error below 3e-4, ample for
-// operands that are rounded to bf16 next. Runs on the FMA pipe, leaving the
-// exponential unit to the exponentials.
-__device__ __forceinline__ float rcp_newton(float x) {
-  float y = __int_as_float(0x7EF311C7 - __float_as_int(x));
-  y = y * fmaf(-x, y, 2.0f);
-  y = y * fmaf(-x, y, 2.0f);
+// 1/x for normal positive x: the hardware approximate reciprocal (a single
+// special-function instruction, error a few ulp), ample for operands that
+// are rounded to bf16 or tf32 next.
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
@@ -410,7 +407,7 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         kr[i] = __ldg(reinterpret_cast<const unsigned int*>(k + tok * DK + c0));
         qr[i] = __ldg(reinterpret_cast<const unsigned int*>(q + tok * DK + c0));
         vr[i] = __ldg(reinterpret_cast<const unsigned int*>(v + tok * DV + c0));
-        bt[i] = __ldg(beta + tok);
+        if ((warp & 1) == 0) bt[i] = __ldg(beta + tok);   // only pr == 0 stores beta
       }
     }
   };
@@ -556,7 +553,7 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         const float k0 = __uint_as_float(kr[i] << 16), k1 = __uint_as_float(kr[i] & 0xffff0000u);
         const float q0 = __uint_as_float(qr[i] << 16), q1 = __uint_as_float(qr[i] & 0xffff0000u);
         const float f0 = __expf(g0[i] - mid0[a]), f1 = __expf(g1[i] - mid1[a]);
-        const float fi0 = rcp_newton(f0), fi1 = rcp_newton(f1);
+        const float fi0 = rcp_approx(f0), fi1 = rcp_approx(f1);
         *reinterpret_cast<uint32_t*>(pAGk + ro) = pack_bf16x2(k0 * f0, k1 * f1);
         *reinterpret_cast<uint32_t*>(pAGk + ro + 8192) = pack_bf16x2(q0 * f0, q1 * f1);
         const float e0 = k0 * fi0, e1 = k1 * fi1;
@@ -581,13 +578,18 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         kt_c1[i] = e1 * kt1[a];
       }
       // K~ as a K-major tf32 operand [c][j]: positions 16 a + 2 rg, +1 per channel.
+      // Lanes 4-7 of every 8 store their second channel first: the 8 lanes of
+      // a store then write rows c = 0..7 (mod 8), i.e. all eight 16-byte
+      // positions of the swizzle (no bank conflicts).
+      const int odd = (lane >> 2) & 1;
 #pragma unroll
       for (int a = 0; a < 4; ++a) {
         const int j = 16 * a + 2 * rg;
-        *reinterpret_cast<float2*>(smem + OFF_KT + tc::sw128<4>(c0, j, 128)) =
-            make_float2(kt_c0[2 * a], kt_c0[2 * a + 1]);
-        *reinterpret_cast<float2*>(smem + OFF_KT + tc::sw128<4>(c0 + 1, j, 128)) =
-            make_float2(kt_c1[2 * a], kt_c1[2 * a + 1]);
+        const float2 v0 = make_float2(kt_c0[2 * a], kt_c0[2 * a + 1]);
+        const float2 v1 = make_float2(kt_c1[2 * a], kt_c1[2 * a + 1]);
+        *reinterpret_cast<float2*>(smem + OFF_KT + tc::sw128<4>(c0 + odd, j, 128)) = odd ? v1 : v0;
+        *reinterpret_cast<float2*>(smem + OFF_KT + tc::sw128<4>(c0 + 1 - odd, j, 128)) =
+            odd ? v0 : v1;
       }
     }
     tc::fence_async_smem();

@@ -32,6 +32,8 @@
 
 namespace kda {
 
+bool chunk_pointers_aligned(const void* q, const void* k, const void* v, const float* la,
+                            const void* o, const float* sT);
 cudaError_t launch_chunk64(const void* q, const void* k, const void* v, const float* la,
                            const float* beta, const float* s0, const int32_t* cu, int n_seq,
                            int T, int H, void* o, float* sT, int32_t* order,
@@ -80,6 +82,8 @@ extern "C" kda_status kda_prefill_noalloc(const void* q, const void* k, const vo
   if (T > 0 && (!q || !k || !v || !log_alpha || !beta || !o)) return KDA_ERR_INVALID_ARG;
   if ((long long)T * H * 128 >= (1LL << 40)) return KDA_ERR_UNSUPPORTED;
   if ((long long)n_seq * H * 4 > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+  if (T > 0 && !kda::chunk_pointers_aligned(q, k, v, log_alpha, o, final_state))
+    return KDA_ERR_INVALID_ARG;
   if (n_seq == 0) return KDA_OK;
   int32_t* scratch = nullptr;
   if (kda::noalloc::scratch_for_current_device(&scratch) != cudaSuccess) return KDA_ERR_CUDA;

@@ -101,6 +101,9 @@ size_t kda_prefill_workspace_bytes(int n_seq, int has_cu_seqlens);
  *   dk = dv = 128). With dtype KDA_F32 the recurrent kernel always runs.
  * final_state may alias init_state (each chain reads its initial state
  *   before writing its final one). o must not alias any input.
+ * The chunked kernel needs q, k, v, o, log_alpha and final_state 16-byte
+ *   aligned (it moves them in 8- and 16-byte vectors); otherwise
+ *   KDA_ERR_INVALID_ARG and nothing is launched.
  * workspace: at least kda_prefill_workspace_bytes(n_seq, cu_seqlens != NULL)
  *   bytes of device memory, 256-byte aligned; may be NULL when that is 0.
  */
@@ -144,7 +147,7 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v,
  * (bf16); beta [T, H]; cu_seqlens int32 [n_seq + 1]; init_state and
  * final_state [n_seq, H, 128, 128] fp32 or NULL.
  * Limits: n_seq <= KDA_NOALLOC_MAX_SEQS, else KDA_ERR_UNSUPPORTED and
- * nothing is launched. The fixed scratch (256 KiB per device, held until the
+ * nothing is launched; pointers aligned as kda_prefill's chunked path needs. The fixed scratch (256 KiB per device, held until the
  * process exits) is shared by every call on a device, so calls whose work
  * overlaps on the GPU race on it; calls on one stream are ordered and safe.
  * The first call on a device looks up the scratch's device address (once per

@@ -74,6 +74,11 @@ def _prefill(**kw):
     (dict(cu=FAKE, n_seq=4), kda.KDA_ERR_WORKSPACE),       # varlen needs its workspace
     (dict(cu=FAKE, n_seq=4, ws=FAKE, ws_bytes=16), kda.KDA_ERR_WORKSPACE),
     (dict(cu=FAKE, n_seq=4, ws=ctypes.c_void_p(0x10004), ws_bytes=256), kda.KDA_ERR_WORKSPACE),
+    # the chunked kernel moves its tensors in 16-byte vectors
+    (dict(la=ctypes.c_void_p(0x10008)), kda.KDA_ERR_INVALID_ARG),
+    (dict(k=ctypes.c_void_p(0x10008)), kda.KDA_ERR_INVALID_ARG),
+    (dict(o=ctypes.c_void_p(0x10002)), kda.KDA_ERR_INVALID_ARG),
+    (dict(sT=ctypes.c_void_p(0x10004)), kda.KDA_ERR_INVALID_ARG),
 ])
 def test_prefill_rejects_bad_arguments(kw, status):
     assert _prefill(**kw) == status

@@ -37,6 +37,13 @@ def test_noalloc_requires_cu_seqlens():
     assert st == kda.KDA_ERR_INVALID_ARG
 
 
+def test_noalloc_rejects_misaligned_tensors():
+    bad = ctypes.c_void_p(0x10008)
+    st = kda.lib().kda_prefill_noalloc(FAKE, FAKE, FAKE, bad, FAKE, None, FAKE, 1, 64, 2,
+                                       FAKE, None, None)
+    assert st == kda.KDA_ERR_INVALID_ARG
+
+
 @pytest.mark.gpu
 def test_noalloc_matches_workspace_entry_point_twice():
     dev = torch.device("cuda")
