@@ -393,22 +393,25 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
   // Inputs of the chunk about to be processed, loaded one chunk ahead.
   float2 lr[8];
   uint32_t kr[8], qr[8], vr[8];
-  float bt[8];
+  float bt[2];   // warp 0 only: beta of rows 2 lane, 2 lane + 1
   auto load_rows = [&](long long tc0, int Lc) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int r = 16 * (i >> 1) + 2 * rg + (i & 1);
       lr[i] = make_float2(0.f, 0.f);
       kr[i] = qr[i] = vr[i] = 0u;
-      bt[i] = 0.f;
       if (r < Lc) {
         const size_t tok = (size_t)(tc0 + r) * H + head;
         lr[i] = __ldg(reinterpret_cast<const float2*>(log_alpha + tok * DK + c0));
         kr[i] = __ldg(reinterpret_cast<const unsigned int*>(k + tok * DK + c0));
         qr[i] = __ldg(reinterpret_cast<const unsigned int*>(q + tok * DK + c0));
         vr[i] = __ldg(reinterpret_cast<const unsigned int*>(v + tok * DV + c0));
-        if ((warp & 1) == 0) bt[i] = __ldg(beta + tok);   // only pr == 0 stores beta
       }
+    }
+    bt[0] = bt[1] = 0.f;
+    if (warp == 0) {
+      if (2 * lane < Lc) bt[0] = __ldg(beta + (size_t)(tc0 + 2 * lane) * H + head);
+      if (2 * lane + 1 < Lc) bt[1] = __ldg(beta + (size_t)(tc0 + 2 * lane + 1) * H + head);
     }
   };
   if (rank < n_chunks) {
@@ -435,10 +438,7 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         s_pair[(a * 8 + rg) * 128 + c0] = l0[2 * a] + l0[2 * a + 1];
         s_pair[(a * 8 + rg) * 128 + c0 + 1] = l1[2 * a] + l1[2 * a + 1];
       }
-      if (pr == 0) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) s_beta[16 * (i >> 1) + 2 * rg + (i & 1)] = bt[i];
-      }
+      if (warp == 0) *reinterpret_cast<float2*>(s_beta + 2 * lane) = make_float2(bt[0], bt[1]);
       __syncthreads();
       {
         // Exclusive scan over rg within each sub-chunk (thread = (a, channel)),
