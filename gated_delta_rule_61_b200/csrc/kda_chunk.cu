@@ -544,7 +544,13 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       uint8_t* const pQT = smem + OFF_QT + sl * 8192u + colb;
       uint8_t* const pBK = smem + OFF_BK + sl * 8192u + colb;
       uint8_t* const pVV = smem + OFF_VV + sl * 8192u + colb;
-      float kt_c0[8], kt_c1[8];
+      // K~ as a K-major tf32 operand [c][j]: positions 16 a + 2 rg, +1 per
+      // channel, stored as soon as both rows of a sub-chunk are done. Lanes
+      // 4-7 of every 8 store their second channel first: the 8 lanes of a
+      // store then write rows c = 0..7 (mod 8), i.e. all eight 16-byte
+      // positions of the swizzle (no bank conflicts).
+      const int odd = (lane >> 2) & 1;
+      float kt_p0 = 0.f, kt_p1 = 0.f;   // the sub-chunk's first row, channels c0, c0 + 1
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int a = i >> 1, e = i & 1;
@@ -574,22 +580,19 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         *reinterpret_cast<uint32_t*>(pQT + ro) = pack_bf16x2(q0 * eg0, q1 * eg1);
         *reinterpret_cast<uint32_t*>(pBK + ro) = pack_bf16x2(k0 * eg0, k1 * eg1);
         *reinterpret_cast<uint32_t*>(pVV + ro) = vr[i];
-        kt_c0[i] = e0 * kt0[a];
-        kt_c1[i] = e1 * kt1[a];
-      }
-      // K~ as a K-major tf32 operand [c][j]: positions 16 a + 2 rg, +1 per channel.
-      // Lanes 4-7 of every 8 store their second channel first: the 8 lanes of
-      // a store then write rows c = 0..7 (mod 8), i.e. all eight 16-byte
-      // positions of the swizzle (no bank conflicts).
-      const int odd = (lane >> 2) & 1;
-#pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        const int j = 16 * a + 2 * rg;
-        const float2 v0 = make_float2(kt_c0[2 * a], kt_c0[2 * a + 1]);
-        const float2 v1 = make_float2(kt_c1[2 * a], kt_c1[2 * a + 1]);
-        *reinterpret_cast<float2*>(smem + OFF_KT + tc::sw128<4>(c0 + odd, j, 128)) = odd ? v1 : v0;
-        *reinterpret_cast<float2*>(smem + OFF_KT + tc::sw128<4>(c0 + 1 - odd, j, 128)) =
-            odd ? v0 : v1;
+        const float kt_e0 = e0 * kt0[a], kt_e1 = e1 * kt1[a];
+        if (e == 0) {
+          kt_p0 = kt_e0;
+          kt_p1 = kt_e1;
+        } else {
+          const int j = 16 * a + 2 * rg;
+          const float2 v0 = make_float2(kt_p0, kt_e0);
+          const float2 v1 = make_float2(kt_p1, kt_e1);
+          *reinterpret_cast<float2*>(smem + OFF_KT + tc::sw128<4>(c0 + odd, j, 128)) =
+              odd ? v1 : v0;
+          *reinterpret_cast<float2*>(smem + OFF_KT + tc::sw128<4>(c0 + 1 - odd, j, 128)) =
+              odd ? v0 : v1;
+        }
       }
     }
     tc::fence_async_smem();
@@ -663,15 +666,18 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       // vv[0..15]: block for the a_lo rows (or the diagonal set), vv[16..31]:
       // block for the a_hi rows. Diagonal entries keep j < r (k rows) or
       // j <= r (q rows).
-      const int lim = is_q ? r + 1 : r;
-      const bool lo_diag = jg == a_lo, hi_diag = jg == a_hi;
+      // Per lane: the source half (vv[16..31] only for a_hi rows off the
+      // diagonal) and how many of the 16 columns survive: all of an R block,
+      // the causal part of the diagonal block (j < r, or j <= r for q rows),
+      // none above it.
+      const int a_row = hi ? a_hi : a_lo;
+      const bool hi_src = hi && jg < a_hi;
+      const int keep = jg < a_row ? 16 : jg == a_row ? (is_q ? r + 1 : r) - 16 * jg : 0;
       float out[16];
 #pragma unroll
       for (int jj = 0; jj < 16; ++jj) {
-        const bool causal = jg * 16 + jj < lim;
-        const float lo = lo_diag ? (causal ? vv[jj] : 0.f) : (jg < a_lo ? vv[jj] : 0.f);
-        const float hv = hi_diag ? (causal ? vv[jj] : 0.f) : (jg < a_hi ? vv[16 + jj] : 0.f);
-        out[jj] = hi ? hv : lo;
+        const float x = hi_src ? vv[16 + jj] : vv[jj];
+        out[jj] = jj < keep ? x : 0.f;
       }
       if (!is_q) {
         const float br = s_beta[r];
