@@ -666,18 +666,32 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       // vv[0..15]: block for the a_lo rows (or the diagonal set), vv[16..31]:
       // block for the a_hi rows. Diagonal entries keep j < r (k rows) or
       // j <= r (q rows).
-      // Per lane: the source half (vv[16..31] only for a_hi rows off the
-      // diagonal) and how many of the 16 columns survive: all of an R block,
-      // the causal part of the diagonal block (j < r, or j <= r for q rows),
-      // none above it.
-      const int a_row = hi ? a_hi : a_lo;
-      const bool hi_src = hi && jg < a_hi;
-      const int keep = jg < a_row ? 16 : jg == a_row ? (is_q ? r + 1 : r) - 16 * jg : 0;
+      // Two equivalent selections; the one that fits each kernel variant's
+      // register budget without spills.
       float out[16];
+      if constexpr (kRing <= 2) {
+        // Per lane: the source half (vv[16..31] only for a_hi rows off the
+        // diagonal) and how many of the 16 columns survive: all of an R block,
+        // the causal part of the diagonal block (j < r, or j <= r for q rows),
+        // none above it.
+        const int a_row = hi ? a_hi : a_lo;
+        const bool hi_src = hi && jg < a_hi;
+        const int keep = jg < a_row ? 16 : jg == a_row ? (is_q ? r + 1 : r) - 16 * jg : 0;
 #pragma unroll
-      for (int jj = 0; jj < 16; ++jj) {
-        const float x = hi_src ? vv[16 + jj] : vv[jj];
-        out[jj] = jj < keep ? x : 0.f;
+        for (int jj = 0; jj < 16; ++jj) {
+          const float x = hi_src ? vv[16 + jj] : vv[jj];
+          out[jj] = jj < keep ? x : 0.f;
+        }
+      } else {
+        const int lim = is_q ? r + 1 : r;
+        const bool lo_diag = jg == a_lo, hi_diag = jg == a_hi;
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+          const bool causal = jg * 16 + jj < lim;
+          const float lo = lo_diag ? (causal ? vv[jj] : 0.f) : (jg < a_lo ? vv[jj] : 0.f);
+          const float hv = hi_diag ? (causal ? vv[jj] : 0.f) : (jg < a_hi ? vv[16 + jj] : 0.f);
+          out[jj] = hi ? hv : lo;
+        }
       }
       if (!is_q) {
         const float br = s_beta[r];
