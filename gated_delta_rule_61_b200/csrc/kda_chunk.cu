@@ -754,23 +754,47 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     }
     const bool receive = kPair && n > 0;
     if (!receive) {
-      const uint32_t tb = tmem + lane_off + TM_S + grp * 32;
-      float s[32];
-      tc::tmem_ld32(tb, s);
-      const int cb = grp * 32;
+      // S -> bf16 tile and in-place decay (16 columns at a time in the
+      // one-CTA variant, where that keeps its registers within budget).
+      if constexpr (kRing == 1) {
 #pragma unroll
-      for (int h8 = 0; h8 < 4; ++h8) {
-        uint32_t p[4];
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint32_t tb = tmem + lane_off + TM_S + grp * 32 + hh * 16;
+          float s[16];
+          tc::tmem_ld16(tb, s);
+          const int cb = grp * 32 + hh * 16;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) p[e] = pack_bf16x2(s[h8 * 8 + 2 * e], s[h8 * 8 + 2 * e + 1]);
-        *reinterpret_cast<uint4*>(smem + OFF_SB + tc::sw128<2>(m, cb + h8 * 8, 128)) =
-            make_uint4(p[0], p[1], p[2], p[3]);
+          for (int h8 = 0; h8 < 2; ++h8) {
+            uint32_t p[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) p[e] = pack_bf16x2(s[h8 * 8 + 2 * e], s[h8 * 8 + 2 * e + 1]);
+            *reinterpret_cast<uint4*>(smem + OFF_SB + tc::sw128<2>(m, cb + h8 * 8, 128)) =
+                make_uint4(p[0], p[1], p[2], p[3]);
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) s[i] *= s_gamma[cb + i];
+          tc::tmem_st16(tb, s);
+        }
+        tc::tmem_wait_st();
+      } else {
+        const uint32_t tb = tmem + lane_off + TM_S + grp * 32;
+        float s[32];
+        tc::tmem_ld32(tb, s);
+        const int cb = grp * 32;
+#pragma unroll
+        for (int h8 = 0; h8 < 4; ++h8) {
+          uint32_t p[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) p[e] = pack_bf16x2(s[h8 * 8 + 2 * e], s[h8 * 8 + 2 * e + 1]);
+          *reinterpret_cast<uint4*>(smem + OFF_SB + tc::sw128<2>(m, cb + h8 * 8, 128)) =
+              make_uint4(p[0], p[1], p[2], p[3]);
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[i] *= s_gamma[cb + i];
+        tc::tmem_st16(tb, s);
+        tc::tmem_st16(tb + 16, s + 16);
+        tc::tmem_wait_st();
       }
-#pragma unroll
-      for (int i = 0; i < 32; ++i) s[i] *= s_gamma[cb + i];
-      tc::tmem_st16(tb, s);
-      tc::tmem_st16(tb + 16, s + 16);
-      tc::tmem_wait_st();
     }
     ok = cta_wait(mbar, phase, 2);
     phase ^= 1;
