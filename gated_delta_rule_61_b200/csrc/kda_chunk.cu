@@ -48,12 +48,17 @@
 //   [128,192) U^T, then D^T = U^T - (W S0)^T   (lane m, column = position)
 //   [192,256) O^T                              (lane m, column = position)
 //   [256,416) Gram result (lanes 0..63 k rows, 64..127 q rows); later W^T
-// Per chunk n: (P1) gates and operand tiles; (P2) Gram MMA, during which the
-// previous chunk's output leaves tensor memory for HBM; (P3) rows of M_kk and
-// M_qk; (P4) block inverse for X on CUDA cores; (P5) W^T and U^T MMAs, during
-// which the state is copied to bf16 and decayed in place; -W to shared
-// memory; (P7) D and the first part of O; (P8) tf32 state update and output
-// correction.
+// Per chunk n: (P1) operand tiles from the chunk's gates and inputs; (P2)
+// Gram MMA, during which the next own chunk's inputs are loaded into
+// registers; (P3) rows of M_kk and M_qk; (P4) block inverse for X in warps
+// 0-7 while warps 8-15 move the previous own chunk's output to HBM; (P5) W^T
+// and U^T MMAs (with one CTA per chain, the state is copied to bf16 and
+// decayed in place meanwhile); -W to shared memory; with a ring, the state
+// is received here; (P7) D and the first part of O, during which the next
+// own chunk's gates (cumulative sums, sub-chunk ends, decay) are formed
+// (with four CTAs per chain, where P7 is on the ring's critical path, at
+// the start of that chunk's P1 instead); (P8) tf32 state update and output
+// correction; with a ring, the state is handed to the next CTA.
 #include "kda_common.cuh"
 #include "kda_tc.cuh"
 
