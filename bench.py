@@ -117,36 +117,55 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
-def dist_setup(n_gpus):
-    import torch
+def dist_setup(n_gpus, backend="nccl"):
+    """Rank layout from the torchrun environment; joins the process group when
+    there is more than one rank (NCCL on the GPUs; gloo for the CPU tests)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
+        import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return world, rank, local
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
+    """The job's time is the slowest rank's: one all-reduce of a scalar."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def barrier(world):
+def barrier(world, sync_cuda=True):
     import torch
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if sync_cuda:
+        torch.cuda.synchronize()
+
+
+def job_value(world, units_per_rank, ms_per_step):
+    """Whole-job throughput: every rank processes units_per_rank per step
+    (independent replicas), the step takes the slowest rank's time."""
+    return world * units_per_rank / (ms_per_step * 1e-3)
+
+
+def rank0_print(rank, line):
+    """The JSON line comes from rank 0 alone."""
+    if rank == 0:
+        print(json.dumps(line), flush=True)
 
 
 def _oracle_sample(n_tok, seed=0):
@@ -186,11 +205,11 @@ def cpu_oracle_prefill(budget_s=12.0, seed=0):
 def bench_reference(args):
     """The fp64 oracle as the reference arm: rank 0 only, each step a bounded
     sample of the workload sized so the whole run takes about two minutes."""
-    import oracle
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    import oracle
     cores = oracle.default_threads()
     per_step = max(0.05, min(args.ref_budget, 120.0 / (args.steps + args.warmup)))
     n_tok = _oracle_tokens_for(per_step, cores)
@@ -216,7 +235,7 @@ def bench_reference(args):
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
-    print(json.dumps(line), flush=True)
+    rank0_print(rank, line)
 
 
 def bench_ours(args):
@@ -262,7 +281,7 @@ def bench_ours(args):
     kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     ms_per_step = total_ms / args.steps
     tokens = P["B"] * P["T"]
-    value = world * tokens / (ms_per_step * 1e-3)
+    value = job_value(world, tokens, ms_per_step)
     head_tokens = tokens * P["H"]
     state_bytes = 2 * P["B"] * P["H"] * P["dk"] * P["dv"] * 4
     alg_bytes = head_tokens * BYTES_PER_HEAD_TOKEN + state_bytes
@@ -468,7 +487,7 @@ def bench_ours(args):
             "decode": dec, "varlen": var, "long": lng, "e2e": e2e, "cpu_baseline": cpu,
             "gpu_launches": args.steps, "clocks": clk.summary(),
         }
-        print(json.dumps(line), flush=True)
+        rank0_print(rank, line)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
