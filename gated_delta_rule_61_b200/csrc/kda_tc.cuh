@@ -176,9 +176,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_wait_ld() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -241,14 +238,6 @@ __device__ __forceinline__ void cluster_sync() {
                ::: "memory");
 }
 
-// Local arrive that also expects `bytes` of asynchronous transactions.
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t saddr, uint32_t bytes) {
-  asm volatile(
-      "{\n\t.reg .b64 st;\n\t"
-      "mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(saddr), "r"(bytes)
-      : "memory");
-}
-
 // Arrive on an mbarrier of another CTA of the cluster (release at cluster scope).
 __device__ __forceinline__ void mbar_remote_arrive(uint32_t cluster_saddr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_saddr)
@@ -274,17 +263,6 @@ __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint32_t saddr, uint32
     if (mbar_try_wait_cluster(saddr, parity)) return true;
     if ((i & 63) == 63 && global_ns() - start > max_ns) return false;
   }
-}
-
-// 16-byte store into another CTA's shared memory that completes 16 bytes of
-// transactions on that CTA's mbarrier.
-__device__ __forceinline__ void st_async_v4(uint32_t cluster_saddr, const float* v,
-                                            uint32_t cluster_mbar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1,%2,%3,%4}, [%5];"
-      ::"r"(cluster_saddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])),
-      "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])), "r"(cluster_mbar)
-      : "memory");
 }
 
 }  // namespace tc
