@@ -43,6 +43,7 @@ FLOPS_PER_HEAD_TOKEN = 6 * 128 * 128 + 2 * 64 * (3 * 128 + 2 * 128)   # dense ti
 PROFILE = os.path.join(ROOT, "profiles", "chunk64_prefill_b4_t8192_h16.txt")
 KERNEL_SRC = os.path.join(ROOT, "gated_delta_rule_61_b200", "csrc", "kda_chunk.cu")
 DECODE_PROFILE = os.path.join(ROOT, "profiles", "decode_step_b256_h32.txt")
+VARLEN_PROFILE = os.path.join(ROOT, "profiles", "chunk64_varlen_64seq_h32.txt")
 DECODE_SRC = os.path.join(ROOT, "gated_delta_rule_61_b200", "csrc", "kda_decode.cu")
 
 
@@ -360,7 +361,8 @@ def bench_ours(args):
                "workload": "KDA packed varlen prefill: 64 sequences log-uniform in [128, 32768] "
                            "(%d tokens, longest %d), H=32, d=128, bf16, C=64" % (t_tot, max(lengths)),
                "roofline": {"bound": "hbm", "achieved": vgbs, "peak": hbm, "unit": "GB/s",
-                            "frac": vgbs / hbm, "traffic": None, "peak_kind": peak_kind},
+                            "frac": vgbs / hbm, "traffic": kernel_traffic(VARLEN_PROFILE),
+                            "peak_kind": peak_kind},
                "gpu_launches_per_step": 2}
         del vin, vo, vs
     # ---------------- long context: one 1M-token prefill, then graph-replayed decode ----------------
