@@ -118,6 +118,19 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return y;
 }
 
+// Read-once inputs: non-coherent loads that do not allocate in L1.
+__device__ __forceinline__ float2 ld_stream_f2(const float* p) {
+  float2 r;
+  asm("ld.global.nc.L1::no_allocate.v2.f32 {%0, %1}, [%2];"
+               : "=f"(r.x), "=f"(r.y) : "l"(p));
+  return r;
+}
+__device__ __forceinline__ uint32_t ld_stream_u32(const __nv_bfloat16* p) {
+  uint32_t r;
+  asm("ld.global.nc.L1::no_allocate.b32 %0, [%1];" : "=r"(r) : "l"(p));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t to_tf32(float x) {
   uint32_t r;
   asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
@@ -407,10 +420,10 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       kr[i] = qr[i] = vr[i] = 0u;
       if (r < Lc) {
         const size_t tok = (size_t)(tc0 + r) * H + head;
-        lr[i] = __ldg(reinterpret_cast<const float2*>(log_alpha + tok * DK + c0));
-        kr[i] = __ldg(reinterpret_cast<const unsigned int*>(k + tok * DK + c0));
-        qr[i] = __ldg(reinterpret_cast<const unsigned int*>(q + tok * DK + c0));
-        vr[i] = __ldg(reinterpret_cast<const unsigned int*>(v + tok * DV + c0));
+        lr[i] = ld_stream_f2(log_alpha + tok * DK + c0);
+        kr[i] = ld_stream_u32(k + tok * DK + c0);
+        qr[i] = ld_stream_u32(q + tok * DK + c0);
+        vr[i] = ld_stream_u32(v + tok * DV + c0);
       }
     }
     bt[0] = bt[1] = 0.f;
