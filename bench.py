@@ -56,14 +56,24 @@ def peaks():
         return 6650.0, 1590.0, "fallback"
 
 
+def code_hash(path):
+    """sha256 (first 16 hex digits) of a CUDA source with comments and
+    whitespace removed: a comment edit keeps it, a code change does not."""
+    import re
+    text = open(path).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    text = re.sub(r"\s+", "", text)
+    return hashlib.sha256(text.encode()).hexdigest()[:16]
+
+
 def kernel_traffic(profile=PROFILE, src=KERNEL_SRC):
     """dram bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source (else None)."""
+    the current kernel code (else None)."""
     try:
         text = open(profile).read()
-        src_hash = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
         fields = dict(line.split(":", 1) for line in text.splitlines() if ":" in line)
-        if fields.get("kernel_source_sha256_16", "").strip() != src_hash:
+        if fields.get("kernel_code_sha256_16", "").strip() != code_hash(src):
             return None
         return int(fields["dram_bytes_per_launch"].strip())
     except Exception:

@@ -137,8 +137,8 @@ __device__ __forceinline__ uint32_t to_tf32(float x) {
   return r;
 }
 
-// Warp-level 16x8x8 tf32 MMA (fp32 accumulate), used for the 32 x 32 block
-// products of the triangular inverse.
+// Warp-level 16x8x8 tf32 MMA (fp32 accumulate), used for the off-diagonal
+// block products of the triangular inverse.
 __device__ __forceinline__ void mma_16x8x8_tf32(float* d, const uint32_t* a, const uint32_t* b) {
   asm volatile(
       "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
@@ -386,7 +386,7 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
   const size_t state_off = ((size_t)seq * H + head) * DK * DV;
 
   // Initial state: S^T[m][c] = S0[c][m]; this warp covers columns [32 grp, +32).
-  // (With a pair, rank 1 receives its first state from rank 0.)
+  // (In a ring, the other CTAs receive their first state from the previous one.)
   if (rank == 0) {
     float vals[32];
 #pragma unroll
