@@ -5,3 +5,4 @@
 #include "kda_recurrent.cu"
 #include "kda_chunk.cu"
 #include "kda_noalloc.cu"
+#include "kda_selftest.cu"

@@ -22,7 +22,8 @@ KDA_F32, KDA_BF16 = 0, 1
 CHUNK_LOG_ALPHA_MIN = -10.0
 
 EXPORTS = ("kda_status_string", "kda_version", "kda_prefill_workspace_bytes",
-           "kda_prefill", "kda_decode_step", "kda_prefill_noalloc", "kda_get_device_status")
+           "kda_prefill", "kda_decode_step", "kda_prefill_noalloc", "kda_get_device_status",
+           "kda_selftest_wait_timeout")
 NOALLOC_MAX_SEQS = 65536
 
 
@@ -60,6 +61,8 @@ def lib():
     L.kda_prefill_noalloc.restype = ctypes.c_int
     L.kda_get_device_status.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int), vp]
     L.kda_get_device_status.restype = ctypes.c_int
+    L.kda_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+    L.kda_selftest_wait_timeout.restype = ctypes.c_int
     _lib = L
     return L
 
@@ -217,3 +220,10 @@ def device_status(reset: bool = True, stream=None):
     detail = ctypes.c_int(0)
     st = lib().kda_get_device_status(1 if reset else 0, ctypes.byref(detail), _stream(stream))
     return int(st), int(detail.value)
+
+
+def selftest_wait_timeout(max_ns: int = 2_000_000, stream=None):
+    """Run the bounded-wait failure path on purpose (see
+    kda_selftest_wait_timeout in include/kda.h); returns the launch status.
+    Read the recorded timeout with device_status()."""
+    return int(lib().kda_selftest_wait_timeout(int(max_ns), _stream(stream)))

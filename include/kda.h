@@ -171,6 +171,21 @@ kda_status kda_prefill_noalloc(const void *q, const void *k, const void *v,
  */
 kda_status kda_get_device_status(int reset, int *detail, cudaStream_t stream);
 
+/*
+ * kda_selftest_wait_timeout -- exercise the bounded-wait failure path (a
+ * test hook; the source pages have no counterpart). Launches one tiny kernel
+ * on `stream` whose single thread waits, with the helpers every kernel of the
+ * library uses, on an mbarrier nothing ever arrives on: once with CTA-scope
+ * and once with cluster-scope acquire, each for max_ns nanoseconds of
+ * %globaltimer. Both waits give up and record KDA_ERR_TIMEOUT in the device
+ * status word (detail 9091: both waits, in order), exactly as a kernel
+ * whose MMA or state hand-over never completed would; nothing faults or
+ * traps and the context stays usable. Read the outcome with
+ * kda_get_device_status(1, &detail, stream), which also clears it.
+ *   max_ns  1e3 .. 1e9 (1 us to 1 s), else KDA_ERR_INVALID_ARG.
+ */
+kda_status kda_selftest_wait_timeout(uint64_t max_ns, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
