@@ -298,6 +298,28 @@ def test_golden_unit_key_retrieval():
         np.testing.assert_allclose(S[0], np.array(case["S"]), atol=1e-12, err_msg=case["name"])
 
 
+def test_golden_channel_gate():
+    """Hand-worked values for the channel-wise gate ("Gated Delta Net", "KDA /
+    Kimi Linear"): each key row of the state decays by its own alpha before the
+    key reads it, alpha = 0 clears only its row, and the read-out comes after
+    the write."""
+    with open(os.path.join(GOLDEN, "channel_gate.json")) as f:
+        cases = json.load(f)["cases"]
+    for case in cases:
+        q = np.array(case["q"], dtype=np.float64)[:, None, :]
+        k = np.array(case["k"], dtype=np.float64)[:, None, :]
+        v = np.array(case["v"], dtype=np.float64)[:, None, :]
+        b = np.array(case["beta"], dtype=np.float64)[:, None]
+        with np.errstate(divide="ignore"):
+            la = np.log(np.array(case["alpha"], dtype=np.float64))[:, None, :]   # log 0 = -inf
+        S0 = None
+        if "S0" in case:
+            S0 = np.array(case["S0"], dtype=np.float64)[None, None]
+        o, S = oracle.kda_forward(q, k, v, la, b, init_state=S0)
+        np.testing.assert_allclose(o[:, 0], np.array(case["o"]), atol=1e-12, err_msg=case["name"])
+        np.testing.assert_allclose(S[0, 0], np.array(case["S"]), atol=1e-12, err_msg=case["name"])
+
+
 # ---------------------------------------------------------------------------
 # The pins are sharp: planted mistakes (in Python copies of the loop) fail them
 # ---------------------------------------------------------------------------
