@@ -19,6 +19,18 @@ Pins (tests/test_oracle_pins.py) tie it to what the pages and mathematics
 fix: the no-change, overwrite/retrieval, clear and no-update invariants, the
 unrolled Householder product form, the ungated and gated chunk algebra, and
 split/resume equivalence.
+
+Two further forms of the same recurrence (``kda_forward_ex``):
+  * the gate: per key channel (KDA, section "KDA / Kimi Linear"), one scalar
+    per head and token (section "Gated Delta Net": a data-dependent scalar
+    between 0 and 1 that multiplies the whole previous state) or none
+    (alpha = 1, the plain delta rule of "DeltaNet, or Fast Weight
+    Programmers");
+  * the input prologue of the cached forward in "DeltaNet, or Fast Weight
+    Programmers": q and k pass through SiLU and are L2-normalised over the
+    head dimension (F.normalize, i.e. divided by max(norm, 1e-12)), beta is
+    the sigmoid of its projection; the gate is read as alpha = sigmoid(x) of
+    its projection x (a value between 0 and 1), so log_alpha = log sigmoid(x).
 """
 import ctypes
 import os
@@ -111,6 +123,94 @@ def kda_forward(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None,
     if rc != 0:
         raise RuntimeError("oracle_kda_forward failed with code %d" % rc)
     return o.reshape(out_shape), fin
+
+
+# ---------------------------------------------------------------------------
+# Gate forms and input prologue (plain fp64 numpy, elementwise definitions)
+# ---------------------------------------------------------------------------
+
+GATES = ("channel", "scalar", "none")
+
+
+def expand_gate(log_alpha, gate, tok_head_shape, dk):
+    """The per-key-channel log-decay a gate form stands for, [..., H, dk].
+
+    channel: log_alpha is already [..., H, dk].
+    scalar:  log_alpha is [..., H]; the one decay multiplies the whole state,
+             i.e. the same value on every key channel.
+    none:    alpha = 1 (log_alpha = 0); the argument is ignored.
+    """
+    if gate == "channel":
+        la = _f64(log_alpha)
+        if la.shape != tuple(tok_head_shape) + (dk,):
+            raise ValueError("channel gate must be %s" % ((tuple(tok_head_shape) + (dk,)),))
+        return la
+    if gate == "scalar":
+        la = _f64(log_alpha)
+        if la.shape != tuple(tok_head_shape):
+            raise ValueError("scalar gate must be %s" % (tuple(tok_head_shape),))
+        return np.repeat(la[..., None], dk, axis=-1)
+    if gate == "none":
+        return np.zeros(tuple(tok_head_shape) + (dk,))
+    raise ValueError("gate must be one of %s" % (GATES,))
+
+
+def silu(x):
+    """x * sigmoid(x)."""
+    x = _f64(x)
+    return x * sigmoid(x)
+
+
+def sigmoid(x):
+    """1 / (1 + exp(-x)), evaluated without overflow for either sign."""
+    x = _f64(x)
+    e = np.exp(-np.abs(x))
+    return np.where(x >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+
+
+def log_sigmoid(x):
+    """log(sigmoid(x)) = -log(1 + exp(-x)), evaluated without overflow."""
+    x = _f64(x)
+    return np.minimum(x, 0.0) - np.log1p(np.exp(-np.abs(x)))
+
+
+def l2_normalize(x, eps=1e-12):
+    """x / max(||x||_2, eps) over the last axis."""
+    x = _f64(x)
+    n = np.sqrt(np.sum(x * x, axis=-1, keepdims=True))
+    return x / np.maximum(n, eps)
+
+
+def prologue_qk(x):
+    """A query or key vector from its raw projection: L2-normalised SiLU."""
+    return l2_normalize(silu(x))
+
+
+def kda_forward_ex(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, *,
+                   gate="channel", raw_qk=False, raw_beta=False, raw_gate=False,
+                   n_threads=None):
+    """kda_forward with a gate form and an optional input prologue.
+
+    gate: "channel" (log_alpha [..., H, dk]), "scalar" (log_alpha [..., H]) or
+    "none" (log_alpha ignored). raw_qk: q and k are raw projections and go
+    through prologue_qk; raw_beta: beta holds logits (sigmoid applied);
+    raw_gate: log_alpha holds gate logits x and the decay is log sigmoid(x).
+    The prologue is applied in fp64 before the token loop.
+    """
+    q, k = _f64(q), _f64(k)
+    if raw_qk:
+        q, k = prologue_qk(q), prologue_qk(k)
+    b = _f64(beta)
+    if raw_beta:
+        b = sigmoid(b)
+    la = None
+    if gate != "none":
+        la = _f64(log_alpha)
+        if raw_gate:
+            la = log_sigmoid(la)
+    la = expand_gate(la, gate, q.shape[:-1], q.shape[-1])
+    return kda_forward(q, k, v, la, b, init_state=init_state, cu_seqlens=cu_seqlens,
+                       n_threads=n_threads)
 
 
 def kda_decode_step(q, k, v, log_alpha, beta, state):
