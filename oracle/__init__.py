@@ -53,6 +53,11 @@ def _load():
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             dp, dp, ctypes.c_int]
         lib.oracle_kda_forward.restype = ctypes.c_int
+        lib.oracle_kda_backward.argtypes = [
+            dp, dp, dp, dp, dp, dp, ctypes.POINTER(ctypes.c_int64),
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
+        lib.oracle_kda_backward.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -123,6 +128,48 @@ def kda_forward(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None,
     if rc != 0:
         raise RuntimeError("oracle_kda_forward failed with code %d" % rc)
     return o.reshape(out_shape), fin
+
+
+def kda_backward(q, k, v, log_alpha, beta, d_o, init_state=None, d_final=None,
+                 cu_seqlens=None, n_threads=None):
+    """Reverse mode of kda_forward (same layouts): given dL/do (shaped like o)
+    and dL/dS_final ([N, H, dk, dv] or None = 0), returns a dict with dq, dk,
+    dlog_alpha (shaped like q), dv (like v), dbeta (like beta) and d_init
+    ([N, H, dk, dv]), all fp64."""
+    q, k, v, la, b, g_o = map(_f64, (q, k, v, log_alpha, beta, d_o))
+    s0, g_f = _f64(init_state), _f64(d_final)
+    shapes = dict(q=q.shape, v=v.shape, b=b.shape)
+    if q.ndim == 4:
+        B, T = q.shape[:2]
+        if cu_seqlens is None:
+            cu_seqlens = np.arange(B + 1, dtype=np.int64) * T
+        q, k, v, la, g_o = (x.reshape(B * T, *x.shape[2:]) for x in (q, k, v, la, g_o))
+        b = b.reshape(B * T, -1)
+    T_total, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens is None:
+        cu_seqlens = np.array([0, T_total], dtype=np.int64)
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    n_seq = cu.shape[0] - 1
+    if cu[-1] != T_total or g_o.shape != (T_total, H, dv):
+        raise ValueError("shape mismatch")
+    out = {n: np.zeros((T_total, H, dk)) for n in ("dq", "dk", "dlog_alpha")}
+    out["dv"] = np.zeros((T_total, H, dv))
+    out["dbeta"] = np.zeros((T_total, H))
+    out["d_init"] = np.zeros((n_seq, H, dk, dv))
+    nt = default_threads() if n_threads is None else int(n_threads)
+    rc = _load().oracle_kda_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(s0),
+        cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n_seq, H, dk, dv,
+        _ptr(g_o), _ptr(g_f), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+        _ptr(out["dlog_alpha"]), _ptr(out["dbeta"]), _ptr(out["d_init"]), nt)
+    if rc != 0:
+        raise RuntimeError("oracle_kda_backward failed with code %d" % rc)
+    for n in ("dq", "dk", "dlog_alpha"):
+        out[n] = out[n].reshape(shapes["q"])
+    out["dv"] = out["dv"].reshape(shapes["v"])
+    out["dbeta"] = out["dbeta"].reshape(shapes["b"])
+    return out
 
 
 # ---------------------------------------------------------------------------

@@ -191,3 +191,231 @@ int oracle_kda_forward(const double *q, const double *k, const double *v,
     pthread_mutex_destroy(&job.lock);
     return job.failed ? -2 : 0;
 }
+
+
+/*
+ * Reverse mode of the same recurrence (the gradient a training step needs;
+ * the pages motivate the chunk-wise form as hardware-efficient training,
+ * "DeltaNet, or Parallelizing Linear Transformers with Delta Rule"). For one
+ * chain, given dL/do_t for every token and dL/dS_T, it returns dL/dq_t,
+ * dL/dk_t, dL/dv_t, dL/dlog_alpha_t, dL/dbeta_t and dL/dS_0.
+ *
+ * The forward states are recomputed and kept (T + 1 matrices per chain), then
+ * the tokens are walked backwards with G = dL/dS_t:
+ *     G += q_t do_t^T                 dq_t = S_t do_t            (o_t = S_t^T q_t)
+ *     dd = G^T k_t                    dk_t = G d_t               (S_t = S' + k_t d_t^T)
+ *     dbeta_t = dd . (v_t - r_t)      dv_t = beta_t dd           (d_t = beta_t (v_t - r_t))
+ *     dr = -beta_t dd;  G' = G + k_t dr^T;  dk_t += S' dr         (r_t = S'^T k_t)
+ *     dlog_alpha_t[i] = sum_j S'[i][j] G'[i][j]                   (S' = Diag(exp(la)) S_{t-1})
+ *     G = Diag(alpha_t) G'
+ * and dS_0 is the final G. Plain fp64, one token at a time, sums in index
+ * order; threads over independent (sequence, head) chains.
+ */
+typedef struct {
+    const double *q, *k, *v, *log_alpha, *beta, *init_state, *d_o, *d_final;
+    const int64_t *cu_seqlens;
+    int n_seq, H, dk, dv;
+    double *dq, *dk_out, *dv_out, *dla, *dbeta, *d_init;
+    int next, failed;
+    pthread_mutex_t lock;
+} oracle_bwd_job;
+
+static int run_chain_bwd(oracle_bwd_job *job, int seq, int h)
+{
+    const int H = job->H, dk = job->dk, dv = job->dv;
+    const int64_t t0 = job->cu_seqlens[seq], t1 = job->cu_seqlens[seq + 1];
+    const int64_t L = t1 - t0;
+    const size_t SZ = (size_t)dk * dv;
+    /* states[0] = S_0, states[t + 1] = S after token t0 + t */
+    double *states = (double *)malloc(sizeof(double) * SZ * (size_t)(L + 1));
+    double *G = (double *)malloc(sizeof(double) * SZ);
+    double *Sp = (double *)malloc(sizeof(double) * SZ);
+    double *r = (double *)malloc(sizeof(double) * dv);
+    double *d = (double *)malloc(sizeof(double) * dv);
+    double *dd = (double *)malloc(sizeof(double) * dv);
+    double *dr = (double *)malloc(sizeof(double) * dv);
+    double *alpha = (double *)malloc(sizeof(double) * dk);
+    if (!states || !G || !Sp || !r || !d || !dd || !dr || !alpha) {
+        free(states); free(G); free(Sp); free(r); free(d); free(dd); free(dr); free(alpha);
+        return -1;
+    }
+    const size_t state_off = ((size_t)seq * H + h) * SZ;
+    if (job->init_state)
+        memcpy(states, job->init_state + state_off, sizeof(double) * SZ);
+    else
+        memset(states, 0, sizeof(double) * SZ);
+
+    /* forward, keeping every state */
+    for (int64_t t = 0; t < L; ++t) {
+        const size_t tok = (size_t)(t0 + t) * H + h;
+        const double *kt = job->k + tok * dk, *vt = job->v + tok * dv;
+        const double *lat = job->log_alpha + tok * dk;
+        const double bt = job->beta[tok];
+        double *S = states + (size_t)(t + 1) * SZ;
+        memcpy(S, states + (size_t)t * SZ, sizeof(double) * SZ);
+        for (int a = 0; a < dk; ++a) {
+            const double al = exp(lat[a]);
+            for (int b = 0; b < dv; ++b) S[(size_t)a * dv + b] *= al;
+        }
+        for (int b = 0; b < dv; ++b) {
+            double acc = 0.0;
+            for (int a = 0; a < dk; ++a) acc += S[(size_t)a * dv + b] * kt[a];
+            r[b] = acc;
+        }
+        for (int b = 0; b < dv; ++b) {
+            const double db = bt * (vt[b] - r[b]);
+            for (int a = 0; a < dk; ++a) S[(size_t)a * dv + b] += kt[a] * db;
+        }
+    }
+
+    /* backward */
+    if (job->d_final)
+        memcpy(G, job->d_final + state_off, sizeof(double) * SZ);
+    else
+        memset(G, 0, sizeof(double) * SZ);
+    for (int64_t t = L - 1; t >= 0; --t) {
+        const size_t tok = (size_t)(t0 + t) * H + h;
+        const double *qt = job->q + tok * dk, *kt = job->k + tok * dk, *vt = job->v + tok * dv;
+        const double *lat = job->log_alpha + tok * dk, *dot = job->d_o + tok * dv;
+        const double bt = job->beta[tok];
+        const double *Sprev = states + (size_t)t * SZ, *S = states + (size_t)(t + 1) * SZ;
+        double *dqt = job->dq + tok * dk, *dkt = job->dk_out + tok * dk;
+        double *dvt = job->dv_out + tok * dv, *dlat = job->dla + tok * dk;
+
+        /* recompute S' = Diag(alpha) S_{t-1}, r = S'^T k, d = beta (v - r) */
+        for (int a = 0; a < dk; ++a) {
+            alpha[a] = exp(lat[a]);
+            for (int b = 0; b < dv; ++b) Sp[(size_t)a * dv + b] = alpha[a] * Sprev[(size_t)a * dv + b];
+        }
+        for (int b = 0; b < dv; ++b) {
+            double acc = 0.0;
+            for (int a = 0; a < dk; ++a) acc += Sp[(size_t)a * dv + b] * kt[a];
+            r[b] = acc;
+            d[b] = bt * (vt[b] - r[b]);
+        }
+        /* o_t = S_t^T q_t */
+        for (int a = 0; a < dk; ++a)
+            for (int b = 0; b < dv; ++b) G[(size_t)a * dv + b] += qt[a] * dot[b];
+        for (int a = 0; a < dk; ++a) {
+            double acc = 0.0;
+            for (int b = 0; b < dv; ++b) acc += S[(size_t)a * dv + b] * dot[b];
+            dqt[a] = acc;
+        }
+        /* S_t = S' + k d^T */
+        for (int b = 0; b < dv; ++b) {
+            double acc = 0.0;
+            for (int a = 0; a < dk; ++a) acc += G[(size_t)a * dv + b] * kt[a];
+            dd[b] = acc;
+        }
+        for (int a = 0; a < dk; ++a) {
+            double acc = 0.0;
+            for (int b = 0; b < dv; ++b) acc += G[(size_t)a * dv + b] * d[b];
+            dkt[a] = acc;
+        }
+        /* d = beta (v - r) */
+        double dbt = 0.0;
+        for (int b = 0; b < dv; ++b) {
+            dbt += dd[b] * (vt[b] - r[b]);
+            dvt[b] = bt * dd[b];
+            dr[b] = -bt * dd[b];
+        }
+        job->dbeta[tok] = dbt;
+        /* r = S'^T k: G' = G + k dr^T, dk += S' dr */
+        for (int a = 0; a < dk; ++a) {
+            double acc = 0.0;
+            for (int b = 0; b < dv; ++b) {
+                G[(size_t)a * dv + b] += kt[a] * dr[b];
+                acc += Sp[(size_t)a * dv + b] * dr[b];
+            }
+            dkt[a] += acc;
+        }
+        /* S' = Diag(exp(la)) S_{t-1} */
+        for (int a = 0; a < dk; ++a) {
+            double acc = 0.0;
+            for (int b = 0; b < dv; ++b) acc += Sp[(size_t)a * dv + b] * G[(size_t)a * dv + b];
+            dlat[a] = acc;
+            for (int b = 0; b < dv; ++b) G[(size_t)a * dv + b] *= alpha[a];
+        }
+    }
+    if (job->d_init)
+        memcpy(job->d_init + state_off, G, sizeof(double) * SZ);
+    free(states); free(G); free(Sp); free(r); free(d); free(dd); free(dr); free(alpha);
+    return 0;
+}
+
+static void *worker_bwd(void *arg)
+{
+    oracle_bwd_job *job = (oracle_bwd_job *)arg;
+    const int total = job->n_seq * job->H;
+    for (;;) {
+        pthread_mutex_lock(&job->lock);
+        const int idx = job->next++;
+        pthread_mutex_unlock(&job->lock);
+        if (idx >= total)
+            break;
+        if (run_chain_bwd(job, idx / job->H, idx % job->H) != 0) {
+            pthread_mutex_lock(&job->lock);
+            job->failed = 1;
+            pthread_mutex_unlock(&job->lock);
+        }
+    }
+    return NULL;
+}
+
+/*
+ * oracle_kda_backward: gradients of a loss through oracle_kda_forward.
+ *   inputs as oracle_kda_forward, plus
+ *   d_o      : [T_total, H, dv]     dL/do
+ *   d_final  : [n_seq, H, dk, dv] or NULL (zero)   dL/dS_final
+ *   outputs dq, dk_out, dla : [T_total, H, dk]; dv_out : [T_total, H, dv];
+ *   dbeta : [T_total, H]; d_init : [n_seq, H, dk, dv] or NULL.
+ * Returns 0 on success, -1 on bad arguments, -2 on allocation failure.
+ */
+int oracle_kda_backward(const double *q, const double *k, const double *v,
+                        const double *log_alpha, const double *beta,
+                        const double *init_state, const int64_t *cu_seqlens,
+                        int n_seq, int H, int dk, int dv,
+                        const double *d_o, const double *d_final,
+                        double *dq, double *dk_out, double *dv_out, double *dla,
+                        double *dbeta, double *d_init, int n_threads)
+{
+    if (!q || !k || !v || !log_alpha || !beta || !cu_seqlens || !d_o)
+        return -1;
+    if (!dq || !dk_out || !dv_out || !dla || !dbeta)
+        return -1;
+    if (n_seq < 0 || H <= 0 || dk <= 0 || dv <= 0 || cu_seqlens[0] != 0)
+        return -1;
+    for (int i = 0; i < n_seq; ++i)
+        if (cu_seqlens[i + 1] < cu_seqlens[i])
+            return -1;
+    if (n_threads < 1)
+        n_threads = 1;
+    const int total = n_seq * H;
+    if (n_threads > total)
+        n_threads = total > 0 ? total : 1;
+    oracle_bwd_job job;
+    memset(&job, 0, sizeof(job));
+    job.q = q; job.k = k; job.v = v; job.log_alpha = log_alpha; job.beta = beta;
+    job.init_state = init_state; job.d_o = d_o; job.d_final = d_final;
+    job.cu_seqlens = cu_seqlens; job.n_seq = n_seq; job.H = H; job.dk = dk; job.dv = dv;
+    job.dq = dq; job.dk_out = dk_out; job.dv_out = dv_out; job.dla = dla;
+    job.dbeta = dbeta; job.d_init = d_init;
+    pthread_mutex_init(&job.lock, NULL);
+    pthread_t *tids = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)n_threads);
+    if (!tids) {
+        pthread_mutex_destroy(&job.lock);
+        return -2;
+    }
+    int started = 0;
+    for (int i = 1; i < n_threads; ++i) {
+        if (pthread_create(&tids[i], NULL, worker_bwd, &job) != 0)
+            break;
+        ++started;
+    }
+    worker_bwd(&job);
+    for (int i = 1; i <= started; ++i)
+        pthread_join(tids[i], NULL);
+    free(tids);
+    pthread_mutex_destroy(&job.lock);
+    return job.failed ? -2 : 0;
+}
