@@ -249,6 +249,140 @@ def bench_reference(args):
     rank0_print(rank, line)
 
 
+def _time_calls(fn, n, stream):
+    """Mean device time (ms) of n back-to-back calls, CUDA events on `stream`."""
+    import torch
+    fn()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(n):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / n
+
+
+def bench_forms(args, dev, stream, hbm, world, inp, dec):
+    """The other gate forms (one decay per token, none), the fused input
+    prologue (raw q/k projections, beta and gate logits) and multi-token
+    decode, each on the workload of its base entry point, with its own
+    algorithmic bytes."""
+    import torch
+    from gated_delta_rule_61_b200 import kda
+    from gated_delta_rule_61_b200.inputs import decode_inputs, decode_state
+    P, D = PREFILL, DECODE
+    out = {}
+    head_tokens = P["B"] * P["T"] * P["H"]
+    state_bytes = 2 * P["B"] * P["H"] * P["dk"] * P["dv"] * 4
+    o = torch.empty_like(inp["v"])
+    fs = torch.empty_like(inp["init_state"])
+    g = torch.Generator(device=dev).manual_seed(77)
+    gate_inputs = {
+        "scalar": (torch.nn.functional.logsigmoid(
+            torch.randn(P["B"], P["T"], P["H"], device=dev, generator=g) + 3.0), 4),
+        "none": (None, 0),
+    }
+    for gate, (la, la_bytes) in gate_inputs.items():
+        ms = _time_calls(lambda: kda.prefill(inp["q"], inp["k"], inp["v"], la, inp["beta"],
+                                             init_state=inp["init_state"], chunk=64, gate=gate,
+                                             o=o, final_state=fs, stream=stream), 10, stream)
+        per = 3 * 256 + la_bytes + 4 + 256
+        gbs = (head_tokens * per + state_bytes) / (ms * 1e-3) / 1e9
+        out["prefill_gate_" + gate] = {
+            "ms_per_call": ms, "tokens_per_s": world * P["B"] * P["T"] / (ms * 1e-3),
+            "bytes_per_head_token": per,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": gbs / hbm}}
+    # raw projections: q, k ~ N(0, 1) unnormalised, beta and gate logits
+    raw = {n: torch.randn(inp[n].shape, device=dev, generator=g).to(inp[n].dtype)
+           for n in ("q", "k")}
+    raw["beta"] = torch.randn(inp["beta"].shape, device=dev, generator=g)
+    raw["log_alpha"] = torch.randn(inp["log_alpha"].shape, device=dev, generator=g) + 3.0
+    ms = _time_calls(lambda: kda.prefill(raw["q"], raw["k"], inp["v"], raw["log_alpha"],
+                                         raw["beta"], init_state=inp["init_state"], chunk=64,
+                                         raw_qk=True, raw_beta=True, raw_gate=True, o=o,
+                                         final_state=fs, stream=stream), 10, stream)
+    gbs = (head_tokens * BYTES_PER_HEAD_TOKEN + state_bytes) / (ms * 1e-3) / 1e9
+    out["prefill_raw_inputs"] = {
+        "ms_per_call": ms, "tokens_per_s": world * P["B"] * P["T"] / (ms * 1e-3),
+        "bytes_per_head_token": BYTES_PER_HEAD_TOKEN,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                     "frac": gbs / hbm}}
+    del raw
+    # decode forms and multi-token decode at B=256, H=32
+    S = decode_state(D["B"], D["H"], D["dk"], D["dv"], std=D["std"], seed=17, device=dev)
+    heads = D["B"] * D["H"]
+    sbytes = 2 * D["dk"] * D["dv"] * 4
+    d1 = decode_inputs(D["B"], D["H"], D["dk"], D["dv"], dtype=torch.bfloat16, seed=17,
+                       device=dev)
+    la_s = torch.nn.functional.logsigmoid(torch.randn(D["B"], D["H"], device=dev,
+                                                      generator=g) + 3.0)
+    od = torch.empty(D["B"], D["H"], D["dv"], dtype=torch.bfloat16, device=dev)
+    for name, la, per_la, kw in (("decode_gate_scalar", la_s, 4, dict(gate="scalar")),
+                                 ("decode_raw_inputs", d1["log_alpha"], 512,
+                                  dict(raw_qk=True, raw_beta=True, raw_gate=True))):
+        q1, k1, v1 = (d1[n][:, None] for n in ("q", "k", "v"))
+        la1 = la[:, None]
+        b1 = d1["beta"][:, None]
+        ms = _time_calls(lambda: kda.decode(q1, k1, v1, la1, b1, S, o=od[:, None], stream=stream,
+                                            **kw), 50, stream)
+        per = sbytes + 3 * 256 + per_la + 4 + 256
+        gbs = heads * per / (ms * 1e-3) / 1e9
+        out[name] = {"us_per_step": ms * 1e3, "bytes_per_head_step": per,
+                     "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                                  "frac": gbs / hbm}}
+    single_us = dec["ms_per_step"] * 1e3 if dec else None
+    multi = {}
+    for T in (2, 4, 8, 16):
+        x = {n: torch.randn(D["B"], T, D["H"], D["dk"], device=dev, generator=g).to(torch.bfloat16)
+             for n in ("q", "k", "v")}
+        for n in ("q", "k"):
+            x[n] = (x[n].float() / x[n].float().norm(dim=-1, keepdim=True)).to(torch.bfloat16)
+        la = torch.nn.functional.logsigmoid(torch.randn(D["B"], T, D["H"], D["dk"], device=dev,
+                                                        generator=g) + 3.0)
+        b = torch.sigmoid(torch.randn(D["B"], T, D["H"], device=dev, generator=g))
+        om = torch.empty(D["B"], T, D["H"], D["dv"], dtype=torch.bfloat16, device=dev)
+        ms = _time_calls(lambda: kda.decode(x["q"], x["k"], x["v"], la, b, S, o=om,
+                                            stream=stream), 20, stream)
+        per = sbytes + T * BYTES_PER_HEAD_TOKEN
+        gbs = heads * per / (ms * 1e-3) / 1e9
+        multi["T%d" % T] = {
+            "us_per_call": ms * 1e3, "tokens_per_s": world * D["B"] * T / (ms * 1e-3),
+            "vs_single_steps": (T * single_us / (ms * 1e3)) if single_us else None,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": gbs / hbm}}
+    out["decode_multi_token"] = {
+        "workload": "B=256 H=32 d=128, T tokens per sequence per call, state in place",
+        **multi}
+    # backward of the prefill workload (gradients of every input and the
+    # initial state from dL/do and dL/dS_final)
+    if not args.no_backward:
+        d_o = torch.randn(inp["v"].shape, device=dev, generator=g).to(inp["v"].dtype)
+        d_fin = torch.randn(inp["init_state"].shape, device=dev, generator=g)
+        need = kda.lib().kda_backward_workspace_bytes(P["B"], P["B"] * P["T"], P["H"], P["dk"],
+                                                      P["dv"])
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        ms = _time_calls(lambda: kda.backward(inp["q"], inp["k"], inp["v"], inp["log_alpha"],
+                                              inp["beta"], d_o, init_state=inp["init_state"],
+                                              d_final=d_fin, workspace=ws, stream=stream),
+                         2, stream)
+        # bytes: the forward inputs read twice (checkpoint pass and block
+        # recomputation), d_o, the fp32 gradients written, states
+        per = 2 * (3 * 256 + 512 + 4) + 256 + 4 * (3 * 128 + 128 + 1)
+        gbs = (head_tokens * per + 3 * state_bytes) / (ms * 1e-3) / 1e9
+        out["backward"] = {
+            "workload": "KDA backward of B=4 T=8192 H=16 d=128 bf16 (token-recurrent, "
+                        "checkpoints every 16 tokens)",
+            "ms_per_call": ms, "tokens_per_s": world * P["B"] * P["T"] / (ms * 1e-3),
+            "roofline": {"bound": "latency (serial token chain)", "achieved": gbs,
+                         "peak": hbm, "unit": "GB/s", "frac": gbs / hbm}}
+        del d_o, d_fin, ws
+    del S
+    torch.cuda.empty_cache()
+    return out
+
+
 def bench_ours(args):
     import torch
     from gated_delta_rule_61_b200 import kda
@@ -347,7 +481,8 @@ def bench_ours(args):
                              init_std=0.1, lengths=lengths, device=dev)
         vo = torch.empty_like(vin["v"])
         vs = torch.empty_like(vin["init_state"])
-        ws = torch.empty(kda.workspace_bytes(len(lengths), True), dtype=torch.uint8, device=dev)
+        ws = torch.empty(kda.workspace_bytes(len(lengths), VARLEN["H"], 128, 128, kda.KDA_BF16, 64,
+                                             True), dtype=torch.uint8, device=dev)
 
         def vstep():
             kda.prefill(vin["q"], vin["k"], vin["v"], vin["log_alpha"], vin["beta"],
@@ -441,6 +576,10 @@ def bench_ours(args):
                           "frac": dbytes / (dus * 1e-6) / 1e9 / hbm}}
         del graph, dins, dout, s_work, ls
         torch.cuda.empty_cache()
+    # ---------------- gate forms, fused prologue, multi-token decode ----------------
+    forms = None
+    if not args.no_forms:
+        forms = bench_forms(args, dev, stream, hbm, world, inp, dec)
     clk.__exit__(None, None, None)
 
     # ---------------- end to end through the public API (host buffers) ----------------
@@ -496,7 +635,8 @@ def bench_ours(args):
                          "peak_kind": peak_kind, "kernel_ms": kernel_ms,
                          "tensor": {"achieved_tflops": tflops, "peak_tflops": bf16_tf,
                                     "frac": tflops / bf16_tf}},
-            "decode": dec, "varlen": var, "long": lng, "e2e": e2e, "cpu_baseline": cpu,
+            "decode": dec, "varlen": var, "long": lng, "forms": forms, "e2e": e2e,
+            "cpu_baseline": cpu,
             "gpu_launches": args.steps, "clocks": clk.summary(),
         }
         rank0_print(rank, line)
@@ -516,6 +656,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-varlen", action="store_true")
     ap.add_argument("--no-long", action="store_true")
+    ap.add_argument("--no-forms", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--ref-budget", type=float, default=8.0)

@@ -1,0 +1,318 @@
+// kda_backward.cu -- reverse mode of the KDA recurrence (the gradients a
+// training step needs), token-recurrent with state checkpoints.
+//
+// Pages: "22580: from GPT-2 to Kimi K3, explained", section "DeltaNet, or
+// Parallelizing Linear Transformers with Delta Rule" (the chunk-wise form
+// exists for hardware-efficient training), with the recurrence of "DeltaNet,
+// or Fast Weight Programmers" and the decay of "Gated Delta Net" / "KDA /
+// Kimi Linear". Forward, per token:
+//     S' = Diag(a) S;  r = S'^T k;  d = beta (v - r);  S_t = S' + k d^T;  o = S_t^T q
+// Backward, with G = dL/dS_t (starting from dL/dS_final), per token in
+// reverse:
+//     G += q do^T;             dq = S_t do
+//     dd = G^T k;              dk = G d
+//     dbeta = dd . (v - r);    dv = beta dd;    dr = -beta dd
+//     G' = G + k dr^T;         dk += S' dr
+//     dlog_alpha_i = sum_j S'_ij G'_ij;         G = Diag(a) G'
+// and dL/dS_0 = G at the end.
+//
+// Layout: one CTA per (sequence, head, 32-column slice of dv); thread i owns
+// key row i of the slice's 32 columns of S and of G (registers). Sums over
+// the value columns (dq, dk, dlog_alpha) stay inside a thread; the two sums
+// over key rows per token (r in the recomputation, dd in the reverse step)
+// are a halving-exchange reduction over the warp's lanes plus one shared-
+// memory exchange across warps. Column slices of one head add their partial
+// dq, dk, dlog_alpha and dbeta into the fp32 outputs (red.add; the four
+// slices' order is not fixed, so these gradients can differ between runs in
+// the last bits). dv and dL/dS_0 are written by their slice alone.
+//
+// The states are not stored per token: a first forward pass writes the
+// slice of S at the start of every block of kBlk tokens to the workspace;
+// then, block by block from the last, the block's states are recomputed from
+// its checkpoint into a per-CTA scratch (kBlk x dk x 32 fp32, L2-resident)
+// and walked backwards. S' is recovered as S_t - k d^T with d kept from the
+// recomputation.
+#include "kda_common.cuh"
+
+namespace kda {
+namespace bwd {
+
+constexpr int kBlk = 16;       // tokens per checkpoint block
+constexpr int kCols = 32;      // value columns per CTA
+
+// Halving-exchange sum of 32 per-lane vectors of 32 values over the warp:
+// on return v[0] of lane l holds the warp sum of value l.
+__device__ __forceinline__ float warp_transpose_sum32(float* v, int lane) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const bool up = lane & off;
+#pragma unroll
+    for (int j = 0; j < off; ++j) {
+      const float keep = up ? v[j + off] : v[j];
+      const float send = up ? v[j] : v[j + off];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  return v[0];
+}
+
+__device__ __forceinline__ void red_add(float* p, float x) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(x) : "memory");
+}
+
+template <typename TIn, int DK, int DV>
+__global__ void __launch_bounds__(DK)
+backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
+                const float* __restrict__ log_alpha, const float* __restrict__ beta,
+                const float* __restrict__ init_state, const int32_t* __restrict__ cu_seqlens,
+                const TIn* __restrict__ d_o, const float* __restrict__ d_final, int T, int H,
+                int gate, float* __restrict__ dq, float* __restrict__ dk,
+                float* __restrict__ dv, float* __restrict__ dla, float* __restrict__ dbeta,
+                float* __restrict__ d_init, float* __restrict__ ckpt, float* __restrict__ scratch) {
+  constexpr int kSlices = DV / kCols;
+  constexpr int kWarps = DK / 32;
+  const int slice = blockIdx.x % kSlices;
+  const int head = (blockIdx.x / kSlices) % H;
+  const int seq = blockIdx.x / (kSlices * H);
+  const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
+  const int col0 = slice * kCols;
+
+  long long t_begin, t_end;
+  seq_bounds(cu_seqlens, seq, T, &t_begin, &t_end);
+  const long long len = t_end - t_begin;
+  const int n_blk = (int)((len + kBlk - 1) / kBlk);
+  // This sequence's checkpoint blocks start at floor(t_begin / kBlk) + seq,
+  // which leaves room for ceil(len / kBlk) blocks before the next sequence's.
+  const long long blk0 = t_begin / kBlk + seq;
+  auto ckpt_row = [&](int b) {
+    return ckpt + ((((size_t)(blk0 + b) * H + head) * kSlices + slice) * DK + i) * kCols;
+  };
+  float* scr = scratch + (size_t)blockIdx.x * kBlk * DK * kCols + (size_t)i * kCols;
+
+  __shared__ float s_part[kWarps][kCols];
+  __shared__ float s_d[kBlk][kCols], s_vr[kBlk][kCols];   // d_j and v_j - r_j per token
+
+  const size_t state_off = ((size_t)seq * H + head) * DK * DV + (size_t)i * DV + col0;
+  float S[kCols];
+#pragma unroll
+  for (int j = 0; j < kCols; j += 4) {
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (init_state) x = *reinterpret_cast<const float4*>(init_state + state_off + j);
+    S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
+  }
+
+  // Per-token row inputs of this thread (key row i) and column inputs.
+  auto decay = [&](size_t tok) {
+    return gate == 0 ? expf(__ldg(log_alpha + tok * DK + i))
+         : gate == 1 ? expf(__ldg(log_alpha + tok)) : 1.f;
+  };
+  // One forward step on S (row i, this slice's columns); leaves d_j and
+  // v_j - r_j in s_d[slot], s_vr[slot].
+  auto forward_step = [&](long long t, int slot) {
+    const size_t tok = (size_t)t * H + head;
+    const float a = decay(tok);
+    const float ki = Io<TIn>::load(k + tok * DK + i);
+    float part[kCols];
+#pragma unroll
+    for (int j = 0; j < kCols; ++j) {
+      S[j] *= a;
+      part[j] = S[j] * ki;
+    }
+    const float rl = warp_transpose_sum32(part, lane);
+    s_part[warp][lane] = rl;
+    __syncthreads();
+    const float bt = __ldg(beta + tok);
+    if (warp == 0) {
+      float r = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) r += s_part[w][lane];
+      const float vr = Io<TIn>::load(v + tok * DV + col0 + lane) - r;
+      s_vr[slot][lane] = vr;
+      s_d[slot][lane] = bt * vr;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kCols; ++j) S[j] = fmaf(ki, s_d[slot][j], S[j]);
+  };
+
+  // Pass 1: forward over the sequence, checkpointing S at every block start.
+  for (int b = 0; b < n_blk; ++b) {
+    float* cp = ckpt_row(b);
+#pragma unroll
+    for (int j = 0; j < kCols; j += 4)
+      __stcg(reinterpret_cast<float4*>(cp + j), make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]));
+    const long long tb = t_begin + (long long)b * kBlk;
+    const int nb = (int)((t_end - tb) < kBlk ? (t_end - tb) : kBlk);
+    if (b + 1 < n_blk)
+      for (int s = 0; s < nb; ++s) forward_step(tb + s, 0);
+  }
+
+  // Pass 2: blocks from the last; G = dL/dS.
+  float G[kCols];
+#pragma unroll
+  for (int j = 0; j < kCols; j += 4) {
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (d_final) x = *reinterpret_cast<const float4*>(d_final + state_off + j);
+    G[j] = x.x; G[j + 1] = x.y; G[j + 2] = x.z; G[j + 3] = x.w;
+  }
+  for (int b = n_blk - 1; b >= 0; --b) {
+    const long long tb = t_begin + (long long)b * kBlk;
+    const int nb = (int)((t_end - tb) < kBlk ? (t_end - tb) : kBlk);
+    const float* cp = ckpt_row(b);
+#pragma unroll
+    for (int j = 0; j < kCols; j += 4) {
+      const float4 x = __ldcg(reinterpret_cast<const float4*>(cp + j));
+      S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
+    }
+    // recompute the block, keeping S_t per token in the scratch
+    for (int s = 0; s < nb; ++s) {
+      forward_step(tb + s, s);
+      float* dst = scr + (size_t)s * DK * kCols;
+#pragma unroll
+      for (int j = 0; j < kCols; j += 4)
+        __stcg(reinterpret_cast<float4*>(dst + j), make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]));
+    }
+    // reverse sweep
+    for (int s = nb - 1; s >= 0; --s) {
+      const long long t = tb + s;
+      const size_t tok = (size_t)t * H + head;
+      const float* src = scr + (size_t)s * DK * kCols;
+#pragma unroll
+      for (int j = 0; j < kCols; j += 4) {
+        const float4 x = __ldcg(reinterpret_cast<const float4*>(src + j));
+        S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;   // S_t
+      }
+      const float ki = Io<TIn>::load(k + tok * DK + i);
+      const float qi = Io<TIn>::load(q + tok * DK + i);
+      const float a = decay(tok);
+      const float bt = __ldg(beta + tok);
+      float dov[kCols];
+#pragma unroll
+      for (int j = 0; j < kCols; ++j) dov[j] = Io<TIn>::load(d_o + tok * DV + col0 + j);
+      // o_t = S_t^T q: G += q do^T; dq_i = sum_j S_t,ij do_j
+      float dqi = 0.f;
+      float part[kCols];
+#pragma unroll
+      for (int j = 0; j < kCols; ++j) {
+        dqi = fmaf(S[j], dov[j], dqi);
+        G[j] = fmaf(qi, dov[j], G[j]);
+        part[j] = G[j] * ki;
+      }
+      // dd_j = sum_i G_ij k_i
+      const float ddl = warp_transpose_sum32(part, lane);
+      s_part[warp][lane] = ddl;
+      __syncthreads();
+      float dd[kCols];
+#pragma unroll
+      for (int j = 0; j < kCols; ++j) {
+        float x = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) x += s_part[w][j];
+        dd[j] = x;
+      }
+      // S_t = S' + k d^T; d = beta (v - r); r = S'^T k
+      float dki = 0.f, dlai = 0.f, dbt = 0.f;
+#pragma unroll
+      for (int j = 0; j < kCols; ++j) {
+        const float dj = s_d[s][j];
+        const float sp = fmaf(-ki, dj, S[j]);          // S'_ij
+        const float dr = -bt * dd[j];
+        dki = fmaf(G[j], dj, dki);                     // G d
+        dki = fmaf(sp, dr, dki);                       // S' dr
+        dbt = fmaf(dd[j], s_vr[s][j], dbt);
+        G[j] = fmaf(ki, dr, G[j]);                     // G'
+        dlai = fmaf(sp, G[j], dlai);
+        G[j] *= a;
+      }
+      red_add(dq + tok * DK + i, dqi);
+      red_add(dk + tok * DK + i, dki);
+      if (gate == 0) red_add(dla + tok * DK + i, dlai);
+      if (i == 0) red_add(dbeta + tok, dbt);
+      if (warp == 0) {
+        float x = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) x += s_part[w][lane];
+        dv[tok * DV + col0 + lane] = bt * x;
+      }
+      if (gate == 1) {
+        // one decay per token: sum over the key rows of the CTA
+        float x = dlai;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+        if (lane == 0) red_add(dla + tok, x);
+      }
+      __syncthreads();   // s_part is reused by the next token
+    }
+  }
+  if (d_init) {
+#pragma unroll
+    for (int j = 0; j < kCols; j += 4)
+      *reinterpret_cast<float4*>(d_init + state_off + j) = make_float4(G[j], G[j + 1], G[j + 2], G[j + 3]);
+  }
+}
+
+}  // namespace bwd
+
+// Workspace: checkpoints (floor(tokens / 16) + n_seq + 1 blocks per head, each
+// dk x dv fp32) and one 16 x dk x 32 fp32 scratch per CTA, 256-byte aligned.
+size_t backward_workspace_bytes(int n_seq, long long tokens, int H, int dk, int dv) {
+  if (n_seq <= 0 || H <= 0) return 0;
+  const size_t blocks = (size_t)(tokens / bwd::kBlk) + (size_t)n_seq + 1;
+  const size_t ck = blocks * (size_t)H * dk * dv * sizeof(float);
+  const size_t ctas = (size_t)n_seq * H * (dv / bwd::kCols);
+  const size_t scr = ctas * bwd::kBlk * dk * bwd::kCols * sizeof(float);
+  return (ck + 255) / 256 * 256 + (scr + 255) / 256 * 256;
+}
+
+template <typename TIn, int DK, int DV>
+static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, const float* la,
+                                const float* beta, const float* s0, const int32_t* cu,
+                                const void* d_o, const float* d_final, int n_seq, int T, int H,
+                                int gate, float* dq, float* dk, float* dv, float* dla,
+                                float* dbeta, float* d_init, float* ckpt, float* scratch,
+                                cudaStream_t stream) {
+  const long long blocks = (long long)n_seq * H * (DV / bwd::kCols);
+  bwd::backward_kernel<TIn, DK, DV><<<(unsigned)blocks, DK, 0, stream>>>(
+      (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, s0, cu, (const TIn*)d_o, d_final,
+      T, H, gate, dq, dk, dv, dla, dbeta, d_init, ckpt, scratch);
+  return cudaGetLastError();
+}
+
+// Zeroes the accumulated outputs, then runs the backward kernel.
+cudaError_t launch_backward(const void* q, const void* k, const void* v, const float* la,
+                            const float* beta, const float* s0, const int32_t* cu,
+                            const void* d_o, const float* d_final, int n_seq, int T, int H,
+                            int dk, int dv, bool bf16, int gate, long long tokens, float* dq,
+                            float* dkk, float* dvv, float* dla, float* dbeta, float* d_init,
+                            void* workspace, cudaStream_t stream) {
+  if (n_seq == 0) return cudaSuccess;
+  cudaError_t e;
+  if (tokens > 0) {
+    if ((e = cudaMemsetAsync(dq, 0, sizeof(float) * tokens * H * dk, stream)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(dkk, 0, sizeof(float) * tokens * H * dk, stream)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(dbeta, 0, sizeof(float) * tokens * H, stream)) != cudaSuccess) return e;
+    if (gate != 2) {
+      const size_t n = gate == 0 ? (size_t)tokens * H * dk : (size_t)tokens * H;
+      if ((e = cudaMemsetAsync(dla, 0, sizeof(float) * n, stream)) != cudaSuccess) return e;
+    }
+  }
+  const size_t blocks = (size_t)(tokens / bwd::kBlk) + (size_t)n_seq + 1;
+  const size_t ck = blocks * (size_t)H * dk * dv * sizeof(float);
+  float* ckpt = static_cast<float*>(workspace);
+  float* scratch = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + (ck + 255) / 256 * 256);
+#define KDA_BWD_ARGS q, k, v, la, beta, s0, cu, d_o, d_final, n_seq, T, H, gate, dq, dkk, dvv, dla, \
+                     dbeta, d_init, ckpt, scratch, stream
+  if (bf16) {
+    if (dk == 128 && dv == 128) return launch_bwd_t<__nv_bfloat16, 128, 128>(KDA_BWD_ARGS);
+    if (dk == 128 && dv == 64) return launch_bwd_t<__nv_bfloat16, 128, 64>(KDA_BWD_ARGS);
+    if (dk == 64 && dv == 128) return launch_bwd_t<__nv_bfloat16, 64, 128>(KDA_BWD_ARGS);
+    return launch_bwd_t<__nv_bfloat16, 64, 64>(KDA_BWD_ARGS);
+  }
+  if (dk == 128 && dv == 128) return launch_bwd_t<float, 128, 128>(KDA_BWD_ARGS);
+  if (dk == 128 && dv == 64) return launch_bwd_t<float, 128, 64>(KDA_BWD_ARGS);
+  if (dk == 64 && dv == 128) return launch_bwd_t<float, 64, 128>(KDA_BWD_ARGS);
+  return launch_bwd_t<float, 64, 64>(KDA_BWD_ARGS);
+#undef KDA_BWD_ARGS
+}
+
+}  // namespace kda

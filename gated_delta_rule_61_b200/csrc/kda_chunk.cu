@@ -40,8 +40,9 @@
 // 4 CTAs per chain that take chunks round-robin: each CTA prepares its own
 // chunks (the state-independent work, most of the time) in parallel with the
 // others, and the fp32 state moves to the next CTA through the chain's
-// final_state slot (L2) after each chunk's state update. Warp w reaches tensor-memory lanes
-// [32 (w % 4), +32); the four warps sharing a lane quadrant split the columns.
+// hand-over slot (L2) after each chunk's state update. Warp w reaches
+// tensor-memory lanes [32 (w % 4), +32); the four warps sharing a lane
+// quadrant split the columns.
 // Tensor memory (512 columns, lanes = dv index m for the state-sized
 // accumulators):
 //   [0,128)   S^T (fp32 state, lane m, column c)
@@ -59,6 +60,10 @@
 // (with four CTAs per chain, where P7 is on the ring's critical path, at
 // the start of that chunk's P1 instead); (P8) tf32 state update and output
 // correction; with a ring, the state is handed to the next CTA.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "kda_common.cuh"
 #include "kda_tc.cuh"
 
@@ -88,10 +93,26 @@ constexpr uint32_t OFF_NW = OFF_BG;            // after the solve: -W^T bf16 MN-
 constexpr uint32_t OFF_MISC = 188416;
 constexpr uint32_t MISC_GAMMA = 0, MISC_BETA = 512, MISC_PAIR = 1280,
                    MISC_GF = 17664, MISC_GL = 19712, MISC_MBAR = 21760, MISC_FULL = 21776,
-                   MISC_TMEM = 21784, MISC_TOT4 = 21792;
-constexpr uint32_t kSmemBytes = OFF_MISC + 23840 + 1024;
+                   MISC_TMEM = 21784, MISC_TOT4 = 21792,
+                   MISC_NORM = 23840,   // raw q/k: per-warp partial squared norms [16][16]
+                   MISC_BARA = 24864, MISC_BARB = 24872,   // input-copy mbarriers
+                   MISC_SGATE = 24896;  // scalar gate: one log-decay per row [64]
+constexpr uint32_t kSmemBytes = OFF_MISC + 25152 + 1024;
+// Landing places of the next own chunk's raw inputs (tensor-map copies, 128B
+// swizzled [row][channel] tiles like the operand tiles): k lands in the
+// K e^g tile and q in the Q e^g tile (P1 rewrites both in place), v in its
+// MMA operand tile directly, and log_alpha (four 32-channel boxes of 8 KiB)
+// in the parts of the Gram tiles that are dead from the W/U MMA on (T tile
+// and the tail of A; the solve's scratch in B). k, v and log_alpha are copied
+// as soon as the W/U MMA has read the previous contents, q once the D/O MMA
+// has.
+__device__ __forceinline__ uint32_t lambda_box(int b) {
+  return b == 0 ? OFF_AG + 16384 : b == 1 ? OFF_AG + 24576 : b == 2 ? OFF_BG + 16384
+                                                                     : OFF_BG + 24576;
+}
 // State hand-over between the CTAs of a chain's cluster goes through the
-// chain's final_state slot in global memory (64 KiB, L2-resident): it is
+// chain's hand-over slot in global memory (64 KiB, L2-resident; a workspace
+// region, or the chain's own final_state): it is
 // written and read strictly in turn (CTA r writes S_n+1 after reading S_n;
 // CTA r+1 reads it before writing S_n+2), so one arrive on the reader's
 // mbarrier per hand-over is the only synchronisation needed. While it
@@ -130,6 +151,24 @@ __device__ __forceinline__ uint32_t ld_stream_u32(const __nv_bfloat16* p) {
   asm("ld.global.nc.L1::no_allocate.b32 %0, [%1];" : "=r"(r) : "l"(p));
   return r;
 }
+
+// SiLU from the hardware tanh approximation (one special-function
+// instruction): x * sigmoid(x) = x * (1/2 + tanh(x/2)/2). Its absolute error
+// (about 2.5e-4 |x|) is far below the bf16 rounding the tensor-core operands
+// receive next.
+__device__ __forceinline__ float silu_tanh(float x) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+  return x * fmaf(0.5f, t, 0.5f);
+}
+
+// log(sigmoid(x)) = min(x, 0) - log(1 + e^-|x|); absolute error a few 1e-8
+// (the rounding of 1 + e^-|x|), far below the gate clamp's effect.
+__device__ __forceinline__ float log_sigmoid_fast(float x) {
+  return fminf(x, 0.f) - __logf(1.f + __expf(-fabsf(x)));
+}
+
+__device__ __forceinline__ float sigmoid_fast(float x) { return 1.f / (1.f + __expf(-x)); }
 
 __device__ __forceinline__ uint32_t to_tf32(float x) {
   uint32_t r;
@@ -336,13 +375,22 @@ __device__ __forceinline__ void store_output_8w(uint32_t tmem, uint32_t lane_off
   }
 }
 
-template <int kRing>
+// kGate: 0 = one decay per key channel (log_alpha [.., H, dk]), 1 = one per
+// token (log_alpha [.., H], the same value on every channel), 2 = none.
+// kRawQK: q and k are raw projections; each token's vectors become
+// normalize(silu(x)) here (the row norms are reduced while the gates are
+// formed). flags: bit 1 = beta holds logits (sigmoid applied), bit 2 = the
+// gate holds logits x (log_alpha = log sigmoid(x)).
+template <int kRing, int kGate, bool kRawQK>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                const __nv_bfloat16* __restrict__ v, const float* __restrict__ log_alpha,
                const float* __restrict__ beta, const float* init_state,
                const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ order,
-               int T, int H, __nv_bfloat16* __restrict__ o, float* final_state) {
+               int T, int H, __nv_bfloat16* __restrict__ o, float* final_state, float* xfer,
+               unsigned flags, const __grid_constant__ CUtensorMap tm_q,
+               const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+               const __grid_constant__ CUtensorMap tm_la) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -369,21 +417,29 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     tc::tmem_relinquish();
   }
   const uint32_t mbar_full = sbase + OFF_MISC + MISC_FULL;     // partner's state is in L2
+  const uint32_t bar_a = sbase + OFF_MISC + MISC_BARA;   // k, v, log_alpha landed
+  const uint32_t bar_b = sbase + OFF_MISC + MISC_BARB;   // q landed
   if (tid == 0) {
     tc::mbar_init(mbar, 1);
+    tc::mbar_init(bar_a, 1);
+    tc::mbar_init(bar_b, 1);
     if (kPair) tc::mbar_init(mbar_full, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   cta_sync_tc();
   if (kPair) tc::cluster_sync();   // partner's barriers exist before any remote arrive
   const uint32_t tmem = *tmem_slot;
-  uint32_t phase = 0, full_phase = 0;
+  uint32_t phase = 0, full_phase = 0, phase_a = 0, phase_b = 0;
+  // Thread 0 issues the MMAs and the input copies; on a failed wait it lets
+  // whatever it issued finish (bounded) before memory is released.
+  bool pend_mma = false, pend_a = false, pend_b = false;
   bool ok = true;
 
   const int quad = warp & 3, grp = warp >> 2;
   const int m = quad * 32 + lane;
   const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
   const size_t state_off = ((size_t)seq * H + head) * DK * DV;
+  const size_t xfer_off = state_off;   // this chain's hand-over slot (rings)
 
   // Initial state: S^T[m][c] = S0[c][m]; this warp covers columns [32 grp, +32).
   // (In a ring, the other CTAs receive their first state from the previous one.)
@@ -408,55 +464,108 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
   const int pr = tid & 63, rg = tid >> 6, c0 = 2 * pr;
   float* s_pair = reinterpret_cast<float*>(smem + OFF_MISC + MISC_PAIR);   // [32][128]
   float* s_tot4 = reinterpret_cast<float*>(smem + OFF_MISC + MISC_TOT4);   // [4][128]
-  // Inputs of the chunk about to be processed, loaded one chunk ahead.
-  float2 lr[8];
-  uint32_t kr[8], qr[8], vr[8];
+  // Inputs of a chunk. One thread issues the tensor-map copies of k, v and
+  // log_alpha (bar_a) and of q (bar_b); beta (and a scalar gate) are small
+  // and read with plain loads into registers / shared memory.
   float bt[2];   // warp 0 only: beta of rows 2 lane, 2 lane + 1
-  auto load_rows = [&](long long tc0, int Lc) {
+  float* s_sgate = reinterpret_cast<float*>(smem + OFF_MISC + MISC_SGATE);
+  auto chunk_len = [&](int nn) {
+    const long long tc0 = t_begin + (long long)nn * C;
+    return (int)((t_end - tc0) < C ? (t_end - tc0) : C);
+  };
+  auto issue_kvl = [&](int nn) {
+    const int z = (int)(t_begin + (long long)nn * C);
+    const int Lc = chunk_len(nn);
+    if (tid == 0) {
+      constexpr uint32_t bytes = 2 * 16384u + (kGate == 0 ? 32768u : 0u);
+      tc::mbar_arrive_expect_tx(bar_a, bytes);
+      pend_a = true;
+      tc::tma_load_3d(sbase + OFF_BK, &tm_k, 0, head, z, bar_a);
+      tc::tma_load_3d(sbase + OFF_BK + 8192, &tm_k, 64, head, z, bar_a);
+      tc::tma_load_3d(sbase + OFF_VV, &tm_v, 0, head, z, bar_a);
+      tc::tma_load_3d(sbase + OFF_VV + 8192, &tm_v, 64, head, z, bar_a);
+      if constexpr (kGate == 0) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int r = 16 * (i >> 1) + 2 * rg + (i & 1);
-      lr[i] = make_float2(0.f, 0.f);
-      kr[i] = qr[i] = vr[i] = 0u;
-      if (r < Lc) {
-        const size_t tok = (size_t)(tc0 + r) * H + head;
-        lr[i] = ld_stream_f2(log_alpha + tok * DK + c0);
-        kr[i] = ld_stream_u32(k + tok * DK + c0);
-        qr[i] = ld_stream_u32(q + tok * DK + c0);
-        vr[i] = ld_stream_u32(v + tok * DV + c0);
+        for (int bx = 0; bx < 4; ++bx)
+          tc::tma_load_3d(sbase + lambda_box(bx), &tm_la, 32 * bx, head, z, bar_a);
       }
     }
     bt[0] = bt[1] = 0.f;
     if (warp == 0) {
-      if (2 * lane < Lc) bt[0] = __ldg(beta + (size_t)(tc0 + 2 * lane) * H + head);
-      if (2 * lane + 1 < Lc) bt[1] = __ldg(beta + (size_t)(tc0 + 2 * lane + 1) * H + head);
+      if (2 * lane < Lc) bt[0] = __ldg(beta + (size_t)(z + 2 * lane) * H + head);
+      if (2 * lane + 1 < Lc) bt[1] = __ldg(beta + (size_t)(z + 2 * lane + 1) * H + head);
+    }
+    if constexpr (kGate == 1) {
+      if (warp == 1) {
+        s_sgate[2 * lane] = 2 * lane < Lc ? __ldg(log_alpha + (size_t)(z + 2 * lane) * H + head)
+                                          : 0.f;
+        s_sgate[2 * lane + 1] =
+            2 * lane + 1 < Lc ? __ldg(log_alpha + (size_t)(z + 2 * lane + 1) * H + head) : 0.f;
+      }
+    }
+  };
+  auto issue_q = [&](int nn) {
+    const int z = (int)(t_begin + (long long)nn * C);
+    if (tid == 0) {
+      tc::mbar_arrive_expect_tx(bar_b, 16384u);
+      pend_b = true;
+      tc::tma_load_3d(sbase + OFF_QT, &tm_q, 0, head, z, bar_b);
+      tc::tma_load_3d(sbase + OFF_QT + 8192, &tm_q, 64, head, z, bar_b);
     }
   };
   if (rank < n_chunks) {
-    const long long tf = t_begin + (long long)rank * C;
-    load_rows(tf, (int)((t_end - tf) < C ? (t_end - tf) : C));
+    issue_kvl(rank);
+    issue_q(rank);
+    __syncthreads();   // the scalar gate row is in shared memory
   }
-  // Cumulative gates of a chunk from the prefetched log_alpha rows (lr):
+  // Cumulative gates of a chunk from its landed log_alpha tile (after bar_a):
   // pair sums per (sub-chunk, rg) -> one exclusive scan over the 32 pairs per
   // channel -> each thread adds its own rows. Writes g0/g1 (registers), beta,
   // the first and last g of every sub-chunk and the chunk's decay e^{g_last}
   // to shared memory. Runs for the next chunk while the current chunk's
   // D/O MMA is in flight; it touches no operand tile.
   float g0[8], g1[8];
-  auto gates = [&]() {
+  auto gates = [&](int Lc) -> bool {
     {
+      if (!cta_wait(bar_a, phase_a, 6)) return false;
+      phase_a ^= 1;
+      pend_a = false;
       float l0[8], l1[8];
+      const bool raw_gate = kGate != 2 && (flags & 4u);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        l0[i] = fmaxf(lr[i].x, kLogAlphaMin);
-        l1[i] = fmaxf(lr[i].y, kLogAlphaMin);
+        const int r = 16 * (i >> 1) + 2 * rg + (i & 1);
+        float x0 = 0.f, x1 = 0.f;   // rows past the chunk's end: no decay
+        if (r < Lc) {
+          if constexpr (kGate == 0) {
+            const float2 lv = *reinterpret_cast<const float2*>(
+                smem + lambda_box(c0 >> 5) + tc::sw128<4>(r, c0 & 31, 64));
+            x0 = lv.x;
+            x1 = lv.y;
+          } else if constexpr (kGate == 1) {
+            x0 = x1 = s_sgate[r];
+          }
+          if (raw_gate) {
+            x0 = log_sigmoid_fast(x0);
+            x1 = kGate == 1 ? x0 : log_sigmoid_fast(x1);
+          }
+        }
+        l0[i] = fmaxf(x0, kLogAlphaMin);
+        l1[i] = fmaxf(x1, kLogAlphaMin);
       }
 #pragma unroll
       for (int a = 0; a < 4; ++a) {
         s_pair[(a * 8 + rg) * 128 + c0] = l0[2 * a] + l0[2 * a + 1];
         s_pair[(a * 8 + rg) * 128 + c0 + 1] = l1[2 * a] + l1[2 * a + 1];
       }
-      if (warp == 0) *reinterpret_cast<float2*>(s_beta + 2 * lane) = make_float2(bt[0], bt[1]);
+      if (warp == 0) {
+        float b0 = bt[0], b1 = bt[1];
+        if (flags & 2u) {   // logits; rows past the chunk's end keep beta = 0
+          b0 = 2 * lane < Lc ? sigmoid_fast(b0) : 0.f;
+          b1 = 2 * lane + 1 < Lc ? sigmoid_fast(b1) : 0.f;
+        }
+        *reinterpret_cast<float2*>(s_beta + 2 * lane) = make_float2(b0, b1);
+      }
       __syncthreads();
       {
         // Exclusive scan over rg within each sub-chunk (thread = (a, channel)),
@@ -506,16 +615,69 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       }
     }
     __syncthreads();
+    return true;
   };
-  if (rank < n_chunks) gates();
+  if (rank < n_chunks) ok = gates(chunk_len(rank));
 
-  for (int n = rank; n < n_chunks; n += step) {
+  for (int n = rank; ok && n < n_chunks; n += step) {
     const long long t0 = t_begin + (long long)n * C;
+    const int L = chunk_len(n);
+    // This thread's two channels of row slot i of a landed bf16 tile (raw k
+    // or q), zero past the chunk's end.
+    const uint32_t sw_rbase = (uint32_t)((rg >> 2) * 1024 + (rg & 3) * 256 + (c0 & 7) * 2);
+    auto raw_pair = [&](uint32_t tile, int i) -> uint32_t {
+      const int a = i >> 1, e = i & 1;
+      const int r = 16 * a + 2 * rg + e;
+      const uint32_t off = (uint32_t)(c0 >> 6) * 8192u + sw_rbase + (uint32_t)(a * 2048 + e * 128) +
+                           ((uint32_t)(((c0 & 63) >> 3) ^ (2 * (rg & 3) + e)) << 4);
+      return r < L ? *reinterpret_cast<const uint32_t*>(smem + tile + off) : 0u;
+    };
 
     // ---- P1: operand tiles. The gates were formed during the previous own
     // chunk's D/O MMA, except with four CTAs per chain, where that MMA is on
     // the chain's critical path and the gates are formed here. -----------
-    if (kRing > 2 && n != rank) gates();
+    if (kRing > 2 && n != rank) {
+      ok = gates(L);
+      if (!ok) break;
+    }
+    ok = cta_wait(bar_b, phase_b, 7);   // q of this chunk has landed
+    if (!ok) break;
+    phase_b ^= 1;
+    pend_b = false;
+    if constexpr (kRawQK) {
+      // Squared norms of SiLU(k) and SiLU(q) per row: this thread's two
+      // channels, reduced over the warp's 32 lanes by halving exchanges
+      // (16 values in 16 shuffles: at each level a lane keeps the half of
+      // its values selected by its lane bit and adds the partner's copy of
+      // that half), so lane l ends with the warp sum of value (l >> 1) & 15;
+      // the two warps of a row group are added when the tiles are built.
+      float nv[16];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t kr = raw_pair(OFF_BK, i), qr = raw_pair(OFF_QT, i);
+        const float k0 = silu_tanh(__uint_as_float(kr << 16));
+        const float k1 = silu_tanh(__uint_as_float(kr & 0xffff0000u));
+        const float q0 = silu_tanh(__uint_as_float(qr << 16));
+        const float q1 = silu_tanh(__uint_as_float(qr & 0xffff0000u));
+        nv[i] = fmaf(k0, k0, k1 * k1);
+        nv[8 + i] = fmaf(q0, q0, q1 * q1);
+      }
+#pragma unroll
+      for (int off = 16; off >= 2; off >>= 1) {
+        const bool up = lane & off;
+#pragma unroll
+        for (int j = 0; j < off / 2; ++j) {
+          const float keep = up ? nv[j + off / 2] : nv[j];
+          const float send = up ? nv[j] : nv[j + off / 2];
+          nv[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+      }
+      nv[0] += __shfl_xor_sync(0xffffffffu, nv[0], 1);
+      const int idx = (lane >> 1) & 15;
+      float* s_norm = reinterpret_cast<float*>(smem + OFF_MISC + MISC_NORM);
+      if ((lane & 1) == 0) s_norm[warp * 16 + idx] = nv[0];
+      __syncthreads();
+    }
     {
       // Sub-chunk midpoints m_a and the per-channel factors, from five
       // exponentials per channel: e^{m_0}, e^{m_a - m_(a-1)} and e^{g_last - m_3};
@@ -561,7 +723,6 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       uint8_t* const pBGe = smem + OFF_BG + sl * 20480u + colb;
       uint8_t* const pQT = smem + OFF_QT + sl * 8192u + colb;
       uint8_t* const pBK = smem + OFF_BK + sl * 8192u + colb;
-      uint8_t* const pVV = smem + OFF_VV + sl * 8192u + colb;
       // K~ as a K-major tf32 operand [c][j]: positions 16 a + 2 rg, +1 per
       // channel, stored as soon as both rows of a sub-chunk are done. Lanes
       // 4-7 of every 8 store their second channel first: the 8 lanes of a
@@ -574,30 +735,54 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         const int a = i >> 1, e = i & 1;
         const uint32_t ro = (uint32_t)(a * 2048 + e * 128) + (e ? xo1 : xo0);
         // bf16 pairs widen exactly: low half << 16, high half masked.
-        const float k0 = __uint_as_float(kr[i] << 16), k1 = __uint_as_float(kr[i] & 0xffff0000u);
-        const float q0 = __uint_as_float(qr[i] << 16), q1 = __uint_as_float(qr[i] & 0xffff0000u);
+        const uint32_t kr = raw_pair(OFF_BK, i), qr = raw_pair(OFF_QT, i);
+        float k0 = __uint_as_float(kr << 16), k1 = __uint_as_float(kr & 0xffff0000u);
+        float q0 = __uint_as_float(qr << 16), q1 = __uint_as_float(qr & 0xffff0000u);
+        if constexpr (kRawQK) {
+          // normalize(silu(x)): divide by max(|silu(x)|, 1e-12) of the row,
+          // whose squared norm is the sum of the row group's two warps.
+          const float* s_norm = reinterpret_cast<const float*>(smem + OFF_MISC + MISC_NORM);
+          const int w0 = 2 * rg;
+          const float nk = s_norm[w0 * 16 + i] + s_norm[(w0 + 1) * 16 + i];
+          const float nq = s_norm[w0 * 16 + 8 + i] + s_norm[(w0 + 1) * 16 + 8 + i];
+          const float ik = rsqrtf(fmaxf(nk, 1e-24f)), iq = rsqrtf(fmaxf(nq, 1e-24f));
+          k0 = silu_tanh(k0) * ik;
+          k1 = silu_tanh(k1) * ik;
+          q0 = silu_tanh(q0) * iq;
+          q1 = silu_tanh(q1) * iq;
+        }
         const float f0 = __expf(g0[i] - mid0[a]), f1 = __expf(g1[i] - mid1[a]);
         const float fi0 = rcp_approx(f0), fi1 = rcp_approx(f1);
         *reinterpret_cast<uint32_t*>(pAGk + ro) = pack_bf16x2(k0 * f0, k1 * f1);
         *reinterpret_cast<uint32_t*>(pAGk + ro + 8192) = pack_bf16x2(q0 * f0, q1 * f1);
         const float e0 = k0 * fi0, e1 = k1 * fi1;
         *reinterpret_cast<uint32_t*>(pBGe + ro) = pack_bf16x2(e0, e1);
-        // R sets: row 64 + r (a < 1), 80 + r (a < 2), 112 + r (a < 3), scaled
-        // by e^{m_a' - m_a} = product of the dd factors in between.
-        if (a < 1)
-          *reinterpret_cast<uint32_t*>(pBGe + ro + 8192) =
-              pack_bf16x2(e0 * dd0[1], e1 * dd1[1]);
-        if (a < 2)
-          *reinterpret_cast<uint32_t*>(pBGe + ro + 10240) = pack_bf16x2(
-              e0 * (a == 0 ? dd0[1] * dd0[2] : dd0[2]), e1 * (a == 0 ? dd1[1] * dd1[2] : dd1[2]));
-        if (a < 3)
-          *reinterpret_cast<uint32_t*>(pBGe + ro + 14336) = pack_bf16x2(
-              e0 * (a == 0 ? dd0[1] * dd0[2] * dd0[3] : a == 1 ? dd0[2] * dd0[3] : dd0[3]),
-              e1 * (a == 0 ? dd1[1] * dd1[2] * dd1[3] : a == 1 ? dd1[2] * dd1[3] : dd1[3]));
+        // R sets: row 64 + r (set 1), 80 + r (set 2), 112 + r (set 3): k_j
+        // e^{m_a' - g_j} for the later sub-chunks a' > a. The nearest one is
+        // one exponential (at most 1), the farther ones multiply it by dd
+        // factors (each at most 1), so no intermediate underflows while the
+        // product is still representable (starting from E_j, which can be
+        // e^75, lost terms of size e^{g_r - g_j} under strong decay).
+        if (a < 3) {
+          float n0 = k0 * __expf(mid0[a < 3 ? a + 1 : 3] - g0[i]);
+          float n1 = k1 * __expf(mid1[a < 3 ? a + 1 : 3] - g1[i]);
+          const uint32_t set_off = a == 0 ? 8192u : a == 1 ? 10240u : 14336u;
+          *reinterpret_cast<uint32_t*>(pBGe + ro + set_off) = pack_bf16x2(n0, n1);
+          if (a < 2) {
+            n0 *= dd0[a + 2 < 4 ? a + 2 : 3];
+            n1 *= dd1[a + 2 < 4 ? a + 2 : 3];
+            *reinterpret_cast<uint32_t*>(pBGe + ro + (a == 0 ? 10240u : 14336u)) =
+                pack_bf16x2(n0, n1);
+          }
+          if (a < 1) {
+            n0 *= dd0[3];
+            n1 *= dd1[3];
+            *reinterpret_cast<uint32_t*>(pBGe + ro + 14336u) = pack_bf16x2(n0, n1);
+          }
+        }
         const float eg0 = f0 * em0[a], eg1 = f1 * em1[a];
         *reinterpret_cast<uint32_t*>(pQT + ro) = pack_bf16x2(q0 * eg0, q1 * eg1);
         *reinterpret_cast<uint32_t*>(pBK + ro) = pack_bf16x2(k0 * eg0, k1 * eg1);
-        *reinterpret_cast<uint32_t*>(pVV + ro) = vr[i];
         const float kt_e0 = e0 * kt0[a], kt_e1 = e1 * kt1[a];
         if (e == 0) {
           kt_p0 = kt_e0;
@@ -628,14 +813,10 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         tc::mma_bf16_ss(tmem + TM_G, da, db, idesc, ks > 0 ? 1u : 0u);
       }
       tc::mma_commit(mbar);
+      pend_mma = true;
     }
-    // While the Gram MMA runs: load this CTA's next chunk into registers (its
-    // inputs are consumed by then: the gates in the D/O MMA wait, the tiles
-    // in P1) and warm L2 with the chunk after it.
-    if (n + step < n_chunks) {
-      const long long t1 = t0 + (long long)step * C;
-      load_rows(t1, (int)((t_end - t1) < C ? (t_end - t1) : C));
-    }
+    // While the Gram MMA runs: warm L2 with the inputs of the own chunk after
+    // next (the next one's are copied in from P5 on).
     if (n + 2 * step < n_chunks) {
       const long long t1 = t0 + (long long)(2 * step) * C;
       const int row = tid >> 3, part = tid & 7;
@@ -644,17 +825,19 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         if (part < 2) tc::prefetch_l2(q + tok * DK + 64 * part);
         else if (part < 4) tc::prefetch_l2(k + tok * DK + 64 * (part - 2));
         else if (part < 6) tc::prefetch_l2(v + tok * DV + 64 * (part - 4));
-        else tc::prefetch_l2(log_alpha + tok * DK + 64 * (part - 6));
-        if (part == 6) tc::prefetch_l2(log_alpha + tok * DK + 32);
+        else if (kGate == 0) tc::prefetch_l2(log_alpha + tok * DK + 64 * (part - 6));
+        if (kGate == 0 && part == 6) tc::prefetch_l2(log_alpha + tok * DK + 32);
+        if (kGate == 1 && part == 6) tc::prefetch_l2(log_alpha + tok);
         if (part == 7) {
-          tc::prefetch_l2(log_alpha + tok * DK + 96);
+          if (kGate == 0) tc::prefetch_l2(log_alpha + tok * DK + 96);
           tc::prefetch_l2(beta + tok);
         }
       }
     }
     ok = cta_wait(mbar, phase, 1);
-    phase ^= 1;
     if (!ok) break;
+    pend_mma = false;
+    phase ^= 1;
 
     // ---- P3: rows of M_kk (lanes 0..63) and M_qk (lanes 64..127) ---------
     // Warp (quad, grp) assembles columns j in [16 grp, 16 grp + 16) for its 32
@@ -769,6 +952,7 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         tc::mma_bf16_ss(tmem + TM_D, du, dt, idesc, ks > 0 ? 1u : 0u);
       }
       tc::mma_commit(mbar);
+      pend_mma = true;
     }
     const bool receive = kPair && n > 0;
     if (!receive) {
@@ -815,8 +999,12 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       }
     }
     ok = cta_wait(mbar, phase, 2);
-    phase ^= 1;
     if (!ok) break;
+    pend_mma = false;
+    phase ^= 1;
+    // The W/U MMA has read K e^g, V and T: bring in the next own chunk's k,
+    // v and log_alpha (and its beta / scalar gate).
+    if (n + step < n_chunks) issue_kvl(n + step);
     {
       // -W^T to shared memory: lane c holds W^T[c][r]; this warp takes r in [16 grp, +16).
       float w[16];
@@ -832,7 +1020,7 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       }
     }
     if (receive) {
-      // The partner wrote this chunk's entering state to the final_state slot.
+      // The partner wrote this chunk's entering state to the hand-over slot.
       int fail = tc::mbar_wait_cluster_bounded(mbar_full, full_phase, kMaxWaitNs) ? 0 : 1;
       full_phase ^= 1;
       fail = __syncthreads_or(fail);
@@ -843,7 +1031,7 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       }
       float s[32];
       const int cb = grp * 32;
-      const float4* slot = reinterpret_cast<const float4*>(final_state + state_off);
+      const float4* slot = reinterpret_cast<const float4*>(xfer + xfer_off);
 #pragma unroll
       for (int v4 = 0; v4 < 8; ++v4) {
         const float4 x = __ldcg(slot + xfer_chunk(m, cb / 4 + v4));
@@ -882,11 +1070,19 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         tc::mma_bf16_ss(tmem + TM_O, da, dq, id_o, ks > 0 ? 1u : 0u);
       }
       tc::mma_commit(mbar);
+      pend_mma = true;
     }
-    if (kRing <= 2 && n + step < n_chunks) gates();   // next own chunk, while the MMAs run
+    if (kRing <= 2 && n + step < n_chunks) {   // next own chunk, while the MMAs run
+      if (!gates(chunk_len(n + step))) {
+        ok = false;
+        break;
+      }
+    }
     ok = cta_wait(mbar, phase, 3);
-    phase ^= 1;
     if (!ok) break;
+    pend_mma = false;
+    phase ^= 1;
+    if (n + step < n_chunks) issue_q(n + step);   // the O MMA has read Q e^g
 
     // ---- P8: S^T += D^T K~ (tf32, A from TMEM, B K-major); O^T += D^T M_qk^T
     if (tid == 0) {
@@ -903,16 +1099,18 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         tc::mma_tf32_ts(tmem + TM_O, a_t, dm, id_o, 1u);
       }
       tc::mma_commit(mbar);
+      pend_mma = true;
     }
     ok = cta_wait(mbar, phase, 4);
-    phase ^= 1;
     if (!ok) break;
+    pend_mma = false;
+    phase ^= 1;
 
     if (kPair && n + 1 < n_chunks) {
       // Hand the state to the next CTA of the ring, which takes chunk n + 1.
       float s[32];
       tc::tmem_ld32(tmem + lane_off + TM_S + grp * 32, s);
-      float4* slot = reinterpret_cast<float4*>(final_state + state_off);
+      float4* slot = reinterpret_cast<float4*>(xfer + xfer_off);
 #pragma unroll
       for (int v4 = 0; v4 < 8; ++v4)
         __stcg(slot + xfer_chunk(m, grp * 8 + v4),
@@ -944,10 +1142,13 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       final_state[state_off + (size_t)c * DV + m] = s[i];
     }
   }
-  if (!ok) {
-    // A wait gave up: give the outstanding MMAs one more bounded chance to
-    // land before the tensor memory they write is released.
-    if (tid == 0) tc::mbar_wait_bounded(mbar, phase ^ 1, kMaxWaitNs);
+  if (!ok && tid == 0) {
+    // A wait gave up: give outstanding MMAs and input copies one more bounded
+    // chance to land before the tensor and shared memory they write is
+    // released.
+    if (pend_mma) tc::mbar_wait_bounded(mbar, phase, kMaxWaitNs);
+    if (pend_a) tc::mbar_wait_bounded(bar_a, phase_a, kMaxWaitNs);
+    if (pend_b) tc::mbar_wait_bounded(bar_b, phase_b, kMaxWaitNs);
   }
   cta_sync_tc();
   if (kPair) tc::cluster_sync();   // no remote traffic targets this CTA past this point
@@ -974,52 +1175,106 @@ __global__ void identity_order_kernel(int n_seq, int32_t* __restrict__ order) {
     order[i] = i;
 }
 
-}  // namespace chunk64
+// Per-device launch state: the dynamic shared-memory attribute must be set on
+// every device the kernels run on, and the ring choice needs that device's SM
+// count. Set up once per device, under a lock (first calls from several host
+// threads may race).
+struct LaunchState {
+  bool ready;
+  int n_sm;
+};
+constexpr int kMaxDevices = 64;
+static std::mutex g_launch_mutex;
+static LaunchState g_launch[kMaxDevices];
 
-cudaError_t launch_chunk64(const void* q, const void* k, const void* v, const float* la,
-                           const float* beta, const float* s0, const int32_t* cu, int n_seq,
-                           int T, int H, void* o, float* sT, int32_t* order,
-                           cudaStream_t stream) {
-  using namespace chunk64;
-  static bool attr_set = false;
-  static int n_sm = 0;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(chunk64_kernel<1>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
+template <int kGate, bool kRaw>
+static cudaError_t set_smem_attrs() {
+  cudaError_t e = cudaFuncSetAttribute(chunk64_kernel<1, kGate, kRaw>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(chunk64_kernel<2, kGate, kRaw>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(chunk64_kernel<4, kGate, kRaw>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+}
+
+static cudaError_t launch_state_for_current_device(int* n_sm) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_launch_mutex);
+  LaunchState& st = g_launch[dev];
+  if (!st.ready) {
+    if ((e = set_smem_attrs<0, false>()) != cudaSuccess) return e;
+    if ((e = set_smem_attrs<1, false>()) != cudaSuccess) return e;
+    if ((e = set_smem_attrs<2, false>()) != cudaSuccess) return e;
+    if ((e = set_smem_attrs<0, true>()) != cudaSuccess) return e;
+    if ((e = set_smem_attrs<1, true>()) != cudaSuccess) return e;
+    if ((e = set_smem_attrs<2, true>()) != cudaSuccess) return e;
+    int count = 0;
+    e = cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(chunk64_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(chunk64_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    int dev = 0;
-    e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
+    st.n_sm = count;
+    st.ready = true;
   }
-  if (cu && order) {
-    const int blocks = (n_seq + 255) / 256;
-    if (n_seq <= 8192)
-      order_by_length_kernel<<<blocks, 256, 0, stream>>>(cu, n_seq, order);
-    else
-      identity_order_kernel<<<blocks, 256, 0, stream>>>(n_seq, order);
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  const long long chains = (long long)n_seq * H;
-  const __nv_bfloat16* qb = (const __nv_bfloat16*)q;
-  const __nv_bfloat16* kb = (const __nv_bfloat16*)k;
-  const __nv_bfloat16* vb = (const __nv_bfloat16*)v;
-  const int32_t* ord = cu ? order : nullptr;
-  __nv_bfloat16* ob = (__nv_bfloat16*)o;
-  if (sT && 2 * chains <= n_sm) {
-    // Few chains: R = 4 or 2 CTAs per chain (chunks round-robin), all in one
-    // wave; the state passes between them through the final_state slot.
-    const int ring = 4 * chains <= n_sm ? 4 : 2;
+  *n_sm = st.n_sm;
+  return cudaSuccess;
+}
+
+struct ChunkArgs {
+  const __nv_bfloat16 *q, *k, *v;
+  const float *la, *beta, *s0;
+  const int32_t *cu, *order;
+  int T, H;
+  __nv_bfloat16* o;
+  float *sT, *xfer;
+  unsigned flags;
+  CUtensorMap tm_q, tm_k, tm_v, tm_la;
+};
+
+// cuTensorMapEncodeTiled, reached through the runtime's driver entry point
+// (the library does not link the driver library directly). Looked up once.
+static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+static std::once_flag g_encode_once;
+
+static cudaError_t tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
+  std::call_once(g_encode_once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  *fn = g_encode;
+  return g_encode ? cudaSuccess : cudaErrorNotSupported;
+}
+
+// A [tokens][H][128] tensor of bf16 (box 64 channels) or fp32 (box 32
+// channels) as a 3-D tiled map: innermost the channels, then the head, then
+// the token; one box = 64 tokens x 1 head x 128 bytes, 128B-swizzled (the
+// operand tiles' layout); rows past the last token read as zeros.
+static cudaError_t encode_rows(PFN_cuTensorMapEncodeTiled_v12000 fn, CUtensorMap* map,
+                               const void* base, bool bf16, long long tokens, int H) {
+  const cuuint64_t es = bf16 ? 2 : 4;
+  cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)tokens};
+  cuuint64_t strides[2] = {128 * es, (cuuint64_t)H * 128 * es};
+  cuuint32_t box[3] = {bf16 ? 64u : 32u, 1u, 64u};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                        3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int kGate, bool kRaw>
+static cudaError_t launch_variant(const ChunkArgs& a, long long chains, int ring,
+                                  cudaStream_t stream) {
+  if (ring > 1) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(ring * chains));
     cfg.blockDim = dim3(kThreads);
@@ -1033,14 +1288,91 @@ cudaError_t launch_chunk64(const void* q, const void* k, const void* v, const fl
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (ring == 4)
-      return cudaLaunchKernelEx(&cfg, chunk64_kernel<4>, qb, kb, vb, la, beta, s0, cu, ord, T,
-                                H, ob, sT);
-    return cudaLaunchKernelEx(&cfg, chunk64_kernel<2>, qb, kb, vb, la, beta, s0, cu, ord, T, H,
-                              ob, sT);
+      return cudaLaunchKernelEx(&cfg, chunk64_kernel<4, kGate, kRaw>, a.q, a.k, a.v, a.la,
+                                a.beta, a.s0, a.cu, a.order, a.T, a.H, a.o, a.sT, a.xfer,
+                                a.flags, a.tm_q, a.tm_k, a.tm_v, a.tm_la);
+    return cudaLaunchKernelEx(&cfg, chunk64_kernel<2, kGate, kRaw>, a.q, a.k, a.v, a.la,
+                              a.beta, a.s0, a.cu, a.order, a.T, a.H, a.o, a.sT, a.xfer,
+                              a.flags, a.tm_q, a.tm_k, a.tm_v, a.tm_la);
   }
-  chunk64_kernel<1><<<(unsigned)chains, kThreads, kSmemBytes, stream>>>(
-      qb, kb, vb, la, beta, s0, cu, ord, T, H, ob, sT);
+  chunk64_kernel<1, kGate, kRaw><<<(unsigned)chains, kThreads, kSmemBytes, stream>>>(
+      a.q, a.k, a.v, a.la, a.beta, a.s0, a.cu, a.order, a.T, a.H, a.o, a.sT, nullptr, a.flags,
+      a.tm_q, a.tm_k, a.tm_v, a.tm_la);
   return cudaGetLastError();
+}
+
+}  // namespace chunk64
+
+// xfer: a 16-byte aligned buffer of n_seq x H x dk x dv fp32 (laid out like
+// the states) that the CTAs of a ring pass the state through: the caller's
+// workspace, or its final_state (each chain's slot is then its own final
+// state, written last by the owner of the last chunk); NULL runs one CTA per
+// chain. gate: 0 per key channel, 1 scalar per token, 2 none; flags: bit 0
+// raw q/k, bit 1 raw beta, bit 2 raw gate.
+cudaError_t launch_chunk64(const void* q, const void* k, const void* v, const float* la,
+                           const float* beta, const float* s0, const int32_t* cu, int n_seq,
+                           int T, int H, void* o, float* sT, float* xfer, int32_t* order,
+                           int gate, unsigned flags, cudaStream_t stream) {
+  using namespace chunk64;
+  const long long chains = (long long)n_seq * H;
+  int n_sm = 0;
+  cudaError_t e0 = launch_state_for_current_device(&n_sm);
+  if (e0 != cudaSuccess) return e0;
+  if (cu && order) {
+    const int blocks = (n_seq + 255) / 256;
+    if (n_seq <= 8192)
+      order_by_length_kernel<<<blocks, 256, 0, stream>>>(cu, n_seq, order);
+    else
+      identity_order_kernel<<<blocks, 256, 0, stream>>>(n_seq, order);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  ChunkArgs a;
+  a.q = (const __nv_bfloat16*)q;
+  a.k = (const __nv_bfloat16*)k;
+  a.v = (const __nv_bfloat16*)v;
+  a.la = la;
+  a.beta = beta;
+  a.s0 = s0;
+  a.cu = cu;
+  a.order = cu ? order : nullptr;
+  a.T = T;
+  a.H = H;
+  a.o = (__nv_bfloat16*)o;
+  a.sT = sT;
+  a.xfer = xfer;
+  a.flags = flags;
+  // Tensor maps of the token-major inputs: every token of the call (packed:
+  // T; dense batch: n_seq x T).
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  cudaError_t e1 = tensor_map_encoder(&enc);
+  if (e1 != cudaSuccess) return e1;
+  const long long tokens = cu ? (long long)T : (long long)n_seq * T;
+  if (tokens == 0) {
+    memset(&a.tm_q, 0, sizeof(CUtensorMap));   // no chunk to load: never read
+    a.tm_k = a.tm_v = a.tm_la = a.tm_q;
+    return launch_variant<2, false>(a, chains, 1, stream);   // initial -> final states
+  }
+  if ((e1 = encode_rows(enc, &a.tm_q, q, true, tokens, H)) != cudaSuccess) return e1;
+  if ((e1 = encode_rows(enc, &a.tm_k, k, true, tokens, H)) != cudaSuccess) return e1;
+  if ((e1 = encode_rows(enc, &a.tm_v, v, true, tokens, H)) != cudaSuccess) return e1;
+  if (gate == 0) {
+    if ((e1 = encode_rows(enc, &a.tm_la, la, false, tokens, H)) != cudaSuccess) return e1;
+  } else {
+    a.tm_la = a.tm_k;   // not read
+  }
+  // Few chains: R = 4 or 2 CTAs per chain (chunks round-robin), all in one
+  // wave; the state passes between them through the chain's xfer slot.
+  const int ring = (xfer && 2 * chains <= n_sm) ? (4 * chains <= n_sm ? 4 : 2) : 1;
+  const bool raw = flags & 1u;
+  switch (gate) {
+    case 0: return raw ? launch_variant<0, true>(a, chains, ring, stream)
+                       : launch_variant<0, false>(a, chains, ring, stream);
+    case 1: return raw ? launch_variant<1, true>(a, chains, ring, stream)
+                       : launch_variant<1, false>(a, chains, ring, stream);
+    default: return raw ? launch_variant<2, true>(a, chains, ring, stream)
+                        : launch_variant<2, false>(a, chains, ring, stream);
+  }
 }
 
 }  // namespace kda

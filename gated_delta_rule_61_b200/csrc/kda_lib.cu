@@ -4,5 +4,6 @@
 #include "kda_decode.cu"
 #include "kda_recurrent.cu"
 #include "kda_chunk.cu"
+#include "kda_backward.cu"
 #include "kda_noalloc.cu"
 #include "kda_selftest.cu"

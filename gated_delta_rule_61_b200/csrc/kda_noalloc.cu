@@ -22,7 +22,10 @@
 //     one stream, or otherwise ordered, are safe;
 //   - the first call on a device looks up the array's device address (a
 //     runtime call, done once per device with that device current); make
-//     that first call before any stream capture begins.
+//     that first call before any stream capture begins. The address is kept
+//     until the process exits; a cudaDeviceReset of the device unloads the
+//     library's device code and leaves it stale, so the entry point must not
+//     be called on a device that was reset.
 // The kernel writes every entry it later reads (the order kernel fills
 // entries 0..n_seq-1 each call), so nothing has to be cleared between calls.
 #include <mutex>
@@ -36,8 +39,8 @@ bool chunk_pointers_aligned(const void* q, const void* k, const void* v, const f
                             const void* o, const float* sT);
 cudaError_t launch_chunk64(const void* q, const void* k, const void* v, const float* la,
                            const float* beta, const float* s0, const int32_t* cu, int n_seq,
-                           int T, int H, void* o, float* sT, int32_t* order,
-                           cudaStream_t stream);
+                           int T, int H, void* o, float* sT, float* xfer, int32_t* order,
+                           int gate, unsigned flags, cudaStream_t stream);
 
 namespace noalloc {
 
@@ -87,7 +90,10 @@ extern "C" kda_status kda_prefill_noalloc(const void* q, const void* k, const vo
   if (n_seq == 0) return KDA_OK;
   int32_t* scratch = nullptr;
   if (kda::noalloc::scratch_for_current_device(&scratch) != cudaSuccess) return KDA_ERR_CUDA;
+  // With few chains the ring of CTAs hands the state over through each
+  // chain's own final_state slot (no other memory is available here).
   const cudaError_t err = kda::launch_chunk64(q, k, v, log_alpha, beta, init_state, cu_seqlens,
-                                              n_seq, T, H, o, final_state, scratch, stream);
+                                              n_seq, T, H, o, final_state, final_state, scratch,
+                                              0, 0u, stream);
   return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }

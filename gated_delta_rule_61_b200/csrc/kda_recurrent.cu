@@ -8,7 +8,11 @@
 //     o = S^T q = S'^T q + (k . q) d
 // exactly as written (fp32, exact gate, log_alpha = -inf clears). This is the
 // path for fp32 inputs and serves as an independent GPU cross-check of the
-// chunked tensor-core kernel.
+// chunked tensor-core kernel. It takes every gate form (per key channel, one
+// scalar per token as in "Gated Delta Net", or none) and the optional input
+// prologue of the cached forward in "DeltaNet, or Fast Weight Programmers"
+// (SiLU and L2 normalisation of q and k, sigmoid of beta; a gate given as
+// logits x decays by sigmoid(x)).
 //
 // Layout: one CTA per (sequence, head, 32-column slice of dv); 128 threads.
 // Lane j owns value column j of the slice; warp g owns key rows
@@ -25,7 +29,8 @@ recurrent_prefill_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                          const TIn* __restrict__ v, const float* __restrict__ log_alpha,
                          const float* __restrict__ beta, const float* __restrict__ init_state,
                          const int32_t* __restrict__ cu_seqlens, int T, int H,
-                         TIn* __restrict__ o, float* __restrict__ final_state) {
+                         TIn* __restrict__ o, float* __restrict__ final_state, int gate,
+                         unsigned flags) {
   constexpr int kGroups = 4;
   constexpr int RPT = DK / kGroups;     // key rows per thread
   constexpr int kSlices = DV / 32;
@@ -42,7 +47,8 @@ recurrent_prefill_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
 
   __shared__ float s_k[2][DK], s_q[2][DK], s_a[2][DK];
   __shared__ float s_red[2][2][kGroups][32];
-  __shared__ float s_kq[2][kGroups];
+  __shared__ float s_kq[2][kGroups][3];   // k.q and, for raw inputs, |k|^2 and |q|^2
+  const bool raw_qk = flags & kRawQK;
 
   const size_t state_off = ((size_t)seq * H + head) * DK * DV;
   float s[RPT];
@@ -57,7 +63,8 @@ recurrent_prefill_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
     if (threadIdx.x < DK) {
       nk = Io<TIn>::load(k + tok * DK + threadIdx.x);
       nq = Io<TIn>::load(q + tok * DK + threadIdx.x);
-      nla = __ldg(log_alpha + tok * DK + threadIdx.x);
+      nla = gate == kGateChannel ? __ldg(log_alpha + tok * DK + threadIdx.x)
+          : gate == kGateScalar  ? __ldg(log_alpha + tok) : 0.f;
     }
     nv = Io<TIn>::load(v + tok * DV + col);
     nb = __ldg(beta + tok);
@@ -66,17 +73,30 @@ recurrent_prefill_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
 
   for (long long t = t_begin; t < t_end; ++t) {
     const int buf = (int)(t & 1);
-    float kq_part = 0.f;
+    float part[3] = {0.f, 0.f, 0.f};
     if (threadIdx.x < DK) {
-      s_k[buf][threadIdx.x] = nk;
-      s_q[buf][threadIdx.x] = nq;
-      s_a[buf][threadIdx.x] = expf(nla);
-      kq_part = nk * nq;
+      float kk = nk, qq = nq;
+      if (raw_qk) {
+        kk = silu_f(kk);
+        qq = silu_f(qq);
+        part[1] = kk * kk;
+        part[2] = qq * qq;
+      }
+      s_k[buf][threadIdx.x] = kk;
+      s_q[buf][threadIdx.x] = qq;
+      s_a[buf][threadIdx.x] = gate == kGateNone ? 1.f : decay_from(nla, flags);
+      part[0] = kk * qq;
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) kq_part += __shfl_xor_sync(0xffffffffu, kq_part, off);
-    if (lane == 0) s_kq[buf][g] = kq_part;
-    const float vv = nv, bb = nb;
+    for (int j = 0; j < 3; ++j)
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) part[j] += __shfl_xor_sync(0xffffffffu, part[j], off);
+    if (lane == 0) {
+      s_kq[buf][g][0] = part[0];
+      s_kq[buf][g][1] = part[1];
+      s_kq[buf][g][2] = part[2];
+    }
+    const float vv = nv, bb = (flags & kRawBeta) ? sigmoid_f(nb) : nb;
     __syncthreads();
     if (t + 1 < t_end) fetch(t + 1);
 
@@ -93,17 +113,23 @@ recurrent_prefill_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
 
     r = 0.f;
     p = 0.f;
-    float kq = 0.f;
+    float kq = 0.f, nk2 = 0.f, nq2 = 0.f;
 #pragma unroll
     for (int w = 0; w < kGroups; ++w) {
       r += s_red[buf][0][w][lane];
       p += s_red[buf][1][w][lane];
-      kq += s_kq[buf][w];
+      kq += s_kq[buf][w][0];
+      nk2 += s_kq[buf][w][1];
+      nq2 += s_kq[buf][w][2];
     }
-    const float d = bb * (vv - r);
-    if (g == 0) Io<TIn>::store(o + ((size_t)t * H + head) * DV + col, fmaf(kq, d, p));
+    // L2 normalisation of SiLU(k), SiLU(q), folded into the reductions.
+    const float ik = raw_qk ? 1.f / fmaxf(sqrtf(nk2), 1e-12f) : 1.f;
+    const float iq = raw_qk ? 1.f / fmaxf(sqrtf(nq2), 1e-12f) : 1.f;
+    const float d = bb * (vv - r * ik);
+    if (g == 0)
+      Io<TIn>::store(o + ((size_t)t * H + head) * DV + col, fmaf(kq * ik * iq, d, p * iq));
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) s[i] = fmaf(s_k[buf][row0 + i], d, s[i]);
+    for (int i = 0; i < RPT; ++i) s[i] = fmaf(s_k[buf][row0 + i] * ik, d, s[i]);
   }
 
   if (final_state) {
@@ -115,11 +141,12 @@ recurrent_prefill_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
 template <typename TIn, int DK, int DV>
 static cudaError_t launch_rec_t(const void* q, const void* k, const void* v, const float* la,
                                 const float* beta, const float* s0, const int32_t* cu,
-                                int n_seq, int T, int H, void* o, float* sT,
-                                cudaStream_t stream) {
+                                int n_seq, int T, int H, void* o, float* sT, int gate,
+                                unsigned flags, cudaStream_t stream) {
   const long long blocks = (long long)n_seq * H * (DV / 32);
   recurrent_prefill_kernel<TIn, DK, DV><<<(unsigned)blocks, 128, 0, stream>>>(
-      (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, s0, cu, T, H, (TIn*)o, sT);
+      (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, s0, cu, T, H, (TIn*)o, sT, gate,
+      flags);
   return cudaGetLastError();
 }
 
@@ -127,26 +154,31 @@ template <typename TIn>
 static cudaError_t launch_rec_dtype(const void* q, const void* k, const void* v,
                                     const float* la, const float* beta, const float* s0,
                                     const int32_t* cu, int n_seq, int T, int H, int dk,
-                                    int dv, void* o, float* sT, cudaStream_t stream) {
+                                    int dv, void* o, float* sT, int gate, unsigned flags,
+                                    cudaStream_t stream) {
   if (dk == 128 && dv == 128)
-    return launch_rec_t<TIn, 128, 128>(q, k, v, la, beta, s0, cu, n_seq, T, H, o, sT, stream);
+    return launch_rec_t<TIn, 128, 128>(q, k, v, la, beta, s0, cu, n_seq, T, H, o, sT, gate,
+                                       flags, stream);
   if (dk == 128 && dv == 64)
-    return launch_rec_t<TIn, 128, 64>(q, k, v, la, beta, s0, cu, n_seq, T, H, o, sT, stream);
+    return launch_rec_t<TIn, 128, 64>(q, k, v, la, beta, s0, cu, n_seq, T, H, o, sT, gate,
+                                      flags, stream);
   if (dk == 64 && dv == 128)
-    return launch_rec_t<TIn, 64, 128>(q, k, v, la, beta, s0, cu, n_seq, T, H, o, sT, stream);
-  return launch_rec_t<TIn, 64, 64>(q, k, v, la, beta, s0, cu, n_seq, T, H, o, sT, stream);
+    return launch_rec_t<TIn, 64, 128>(q, k, v, la, beta, s0, cu, n_seq, T, H, o, sT, gate,
+                                      flags, stream);
+  return launch_rec_t<TIn, 64, 64>(q, k, v, la, beta, s0, cu, n_seq, T, H, o, sT, gate, flags,
+                                   stream);
 }
 
 cudaError_t launch_recurrent(const void* q, const void* k, const void* v, const float* la,
                              const float* beta, const float* s0, const int32_t* cu,
                              int n_seq, int T, int H, int dk, int dv, bool bf16, void* o,
-                             float* sT, cudaStream_t stream) {
+                             float* sT, int gate, unsigned flags, cudaStream_t stream) {
   if (n_seq == 0) return cudaSuccess;
   if (bf16)
     return launch_rec_dtype<__nv_bfloat16>(q, k, v, la, beta, s0, cu, n_seq, T, H, dk, dv,
-                                           o, sT, stream);
-  return launch_rec_dtype<float>(q, k, v, la, beta, s0, cu, n_seq, T, H, dk, dv, o, sT,
-                                 stream);
+                                           o, sT, gate, flags, stream);
+  return launch_rec_dtype<float>(q, k, v, la, beta, s0, cu, n_seq, T, H, dk, dv, o, sT, gate,
+                                 flags, stream);
 }
 
 }  // namespace kda

@@ -14,6 +14,7 @@
 //   instruction, so LBO is unused.
 #pragma once
 
+#include <cuda.h>
 #include <stdint.h>
 
 namespace kda {
@@ -178,6 +179,27 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
 
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// ---- tensor-map (TMA) loads into this CTA's shared memory ------------------
+
+// Arm an mbarrier for `bytes` of incoming copies and arrive once (the phase
+// completes when the arrival and all the bytes are in).
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t mbar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes)
+               : "memory");
+}
+
+// One box of a 3-D tiled tensor map at coordinates (x, y, z) (innermost
+// first) into shared memory at dst, completing `box bytes` on mbar. The
+// destination is this CTA's own shared memory; no multicast.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            int z, uint32_t mbar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(mbar)
+      : "memory");
 }
 
 __device__ __forceinline__ void prefetch_l2(const void* p) {

@@ -19,11 +19,16 @@ LIB_PATH = os.path.join(HERE, "libkda.so")
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_ERR_CUDA, \
     KDA_ERR_TIMEOUT = range(6)
 KDA_F32, KDA_BF16 = 0, 1
+KDA_GATE_CHANNEL, KDA_GATE_SCALAR, KDA_GATE_NONE = 0, 1, 2
+KDA_RAW_QK, KDA_RAW_BETA, KDA_RAW_GATE = 1, 2, 4
+GATES = {"channel": KDA_GATE_CHANNEL, "scalar": KDA_GATE_SCALAR, "none": KDA_GATE_NONE}
 CHUNK_LOG_ALPHA_MIN = -10.0
+DECODE_MAX_TOKENS = 16
 
 EXPORTS = ("kda_status_string", "kda_version", "kda_prefill_workspace_bytes",
-           "kda_prefill", "kda_decode_step", "kda_prefill_noalloc", "kda_get_device_status",
-           "kda_selftest_wait_timeout")
+           "kda_prefill", "kda_prefill_ex", "kda_decode_step", "kda_decode_ex",
+           "kda_backward_workspace_bytes", "kda_backward", "kda_prefill_noalloc",
+           "kda_get_device_status", "kda_selftest_wait_timeout")
 NOALLOC_MAX_SEQS = 65536
 
 
@@ -50,13 +55,26 @@ def lib():
     L.kda_status_string.restype = ctypes.c_char_p
     L.kda_version.argtypes = []
     L.kda_version.restype = ctypes.c_int
-    L.kda_prefill_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int]
+    L.kda_prefill_workspace_bytes.argtypes = [ctypes.c_int] * 7
     L.kda_prefill_workspace_bytes.restype = ctypes.c_size_t
     L.kda_prefill.argtypes = [vp, vp, vp, fp, fp, fp, i32p, ip, ip, ip, ip, ip, ip,
                               ctypes.c_int, ctypes.c_int, vp, fp, vp, ctypes.c_size_t, vp]
     L.kda_prefill.restype = ctypes.c_int
+    L.kda_prefill_ex.argtypes = [vp, vp, vp, fp, fp, fp, i32p, ip, ip, ip, ip, ip, ip,
+                                 ctypes.c_int, ctypes.c_int, ctypes.c_uint, ctypes.c_int, vp, fp,
+                                 vp, ctypes.c_size_t, vp]
+    L.kda_prefill_ex.restype = ctypes.c_int
     L.kda_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, ip, ip, ip, ip, ctypes.c_int, vp, vp]
     L.kda_decode_step.restype = ctypes.c_int
+    L.kda_decode_ex.argtypes = [vp, vp, vp, fp, fp, fp, ip, ip, ip, ip, ip, ctypes.c_int,
+                                ctypes.c_int, ctypes.c_uint, vp, vp]
+    L.kda_decode_ex.restype = ctypes.c_int
+    L.kda_backward_workspace_bytes.argtypes = [ip, ctypes.c_int64, ip, ip, ip]
+    L.kda_backward_workspace_bytes.restype = ctypes.c_size_t
+    L.kda_backward.argtypes = [vp, vp, vp, fp, fp, fp, i32p, ip, ip, ip, ip, ip, ip,
+                               ctypes.c_int, ctypes.c_int, vp, fp, fp, fp, fp, fp, fp, fp,
+                               vp, ctypes.c_size_t, vp]
+    L.kda_backward.restype = ctypes.c_int
     L.kda_prefill_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, i32p, ip, ip, ip, vp, fp, vp]
     L.kda_prefill_noalloc.restype = ctypes.c_int
     L.kda_get_device_status.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int), vp]
@@ -99,19 +117,40 @@ def _check(t, name, shape, dtype, device):
         raise ValueError("%s must be contiguous" % name)
 
 
-def workspace_bytes(n_seq: int, has_cu_seqlens: bool) -> int:
-    return int(lib().kda_prefill_workspace_bytes(int(n_seq), 1 if has_cu_seqlens else 0))
+def workspace_bytes(n_seq: int, H: int, dk: int, dv: int, dtype_code: int, chunk: int,
+                    has_cu_seqlens: bool) -> int:
+    """Bytes of workspace kda_prefill needs (see include/kda.h)."""
+    return int(lib().kda_prefill_workspace_bytes(int(n_seq), int(H), int(dk), int(dv),
+                                                 int(dtype_code), int(chunk),
+                                                 1 if has_cu_seqlens else 0))
+
+
+def _flags(raw_qk, raw_beta, raw_gate):
+    return ((KDA_RAW_QK if raw_qk else 0) | (KDA_RAW_BETA if raw_beta else 0)
+            | (KDA_RAW_GATE if raw_gate else 0))
+
+
+def _gate_shape(gate, tok_head):
+    if gate == "channel":
+        return None
+    return tuple(tok_head)
 
 
 def prefill(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, *, chunk=64,
+            gate="channel", raw_qk=False, raw_beta=False, raw_gate=False,
             output_final_state=True, o=None, final_state=None, workspace=None, stream=None):
     """Chunked (chunk=64) or token-recurrent (chunk=0) KDA prefill.
 
-    q, k, log_alpha [B, T, H, dk]; v [B, T, H, dv]; beta [B, T, H];
-    init_state [N, H, dk, dv] or None; cu_seqlens int32 [N+1] (then B = 1).
+    q, k [B, T, H, dk]; v [B, T, H, dv]; beta [B, T, H];
+    log_alpha [B, T, H, dk] (gate "channel"), [B, T, H] ("scalar") or None
+    ("none"); init_state [N, H, dk, dv] or None; cu_seqlens int32 [N+1]
+    (then B = 1). raw_qk / raw_beta / raw_gate: the inputs are raw
+    projections and the kernel applies the prologue (see kda_prefill_ex).
     Returns (o [B, T, H, dv] in q's dtype, final_state [N, H, dk, dv] fp32 or
     None).
     """
+    if gate not in GATES:
+        raise ValueError("gate must be one of %s" % list(GATES))
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dev = q.device
@@ -121,7 +160,12 @@ def prefill(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, *, chunk
     _check(q, "q", (B, T, H, dk), dt, dev)
     _check(k, "k", (B, T, H, dk), dt, dev)
     _check(v, "v", (B, T, H, dv), dt, dev)
-    _check(log_alpha, "log_alpha", (B, T, H, dk), torch.float32, dev)
+    if gate == "channel":
+        _check(log_alpha, "log_alpha", (B, T, H, dk), torch.float32, dev)
+    elif gate == "scalar":
+        _check(log_alpha, "log_alpha", (B, T, H), torch.float32, dev)
+    else:
+        log_alpha = None
     _check(beta, "beta", (B, T, H), torch.float32, dev)
     if init_state is not None:
         _check(init_state, "init_state", (n_seq, H, dk, dv), torch.float32, dev)
@@ -137,17 +181,69 @@ def prefill(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, *, chunk
         final_state = torch.empty((n_seq, H, dk, dv), dtype=torch.float32, device=dev)
     elif final_state is not None:
         _check(final_state, "final_state", (n_seq, H, dk, dv), torch.float32, dev)
-    need = workspace_bytes(n_seq, cu_seqlens is not None) if chunk else 0
+    need = workspace_bytes(n_seq, H, dk, dv, code, chunk, cu_seqlens is not None)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib().kda_prefill(
+    st = lib().kda_prefill_ex(
         _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(init_state),
         _ptr(cu_seqlens), int(n_seq), int(B), int(T), int(H), int(dk), int(dv), code,
-        int(chunk), _ptr(o), _ptr(final_state), _ptr(workspace), ws_bytes, _stream(stream))
+        GATES[gate], _flags(raw_qk, raw_beta, raw_gate), int(chunk), _ptr(o),
+        _ptr(final_state), _ptr(workspace), ws_bytes, _stream(stream))
     if st != KDA_OK:
-        raise KdaError(st, "kda_prefill")
+        raise KdaError(st, "kda_prefill_ex")
     return o, final_state
+
+
+def backward(q, k, v, log_alpha, beta, d_o, init_state=None, cu_seqlens=None, d_final=None,
+             *, gate="channel", workspace=None, stream=None):
+    """Gradients through the recurrence (kda_backward): returns a dict of fp32
+    tensors dq, dk, dv, dlog_alpha (None for gate "none"), dbeta and d_init
+    ([N, H, dk, dv]). Inputs as for prefill (ready inputs, no prologue);
+    d_o shaped like v in v's dtype; d_final [N, H, dk, dv] fp32 or None."""
+    if gate not in GATES:
+        raise ValueError("gate must be one of %s" % list(GATES))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    code = _dtype_code(q)
+    n_seq = B if cu_seqlens is None else cu_seqlens.shape[0] - 1
+    for t, name, shape, dtype in ((q, "q", (B, T, H, dk), dt), (k, "k", (B, T, H, dk), dt),
+                                  (v, "v", (B, T, H, dv), dt), (d_o, "d_o", (B, T, H, dv), dt),
+                                  (beta, "beta", (B, T, H), torch.float32)):
+        _check(t, name, shape, dtype, dev)
+    if gate == "channel":
+        _check(log_alpha, "log_alpha", (B, T, H, dk), torch.float32, dev)
+    elif gate == "scalar":
+        _check(log_alpha, "log_alpha", (B, T, H), torch.float32, dev)
+    else:
+        log_alpha = None
+    for t, name in ((init_state, "init_state"), (d_final, "d_final")):
+        if t is not None:
+            _check(t, name, (n_seq, H, dk, dv), torch.float32, dev)
+    if cu_seqlens is not None:
+        if B != 1:
+            raise ValueError("packed sequences (cu_seqlens) need B == 1")
+        _check(cu_seqlens, "cu_seqlens", (n_seq + 1,), torch.int32, dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = dict(dq=torch.empty(B, T, H, dk, **f32), dk=torch.empty(B, T, H, dk, **f32),
+               dv=torch.empty(B, T, H, dv, **f32), dbeta=torch.empty(B, T, H, **f32),
+               d_init=torch.empty(n_seq, H, dk, dv, **f32))
+    out["dlog_alpha"] = (None if gate == "none" else torch.empty(log_alpha.shape, **f32))
+    need = int(lib().kda_backward_workspace_bytes(int(n_seq), int(B * T), int(H), int(dk),
+                                                  int(dv)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = lib().kda_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(init_state),
+        _ptr(cu_seqlens), int(n_seq), int(B), int(T), int(H), int(dk), int(dv), code,
+        GATES[gate], _ptr(d_o), _ptr(d_final), _ptr(out["dq"]), _ptr(out["dk"]),
+        _ptr(out["dv"]), _ptr(out["dlog_alpha"]), _ptr(out["dbeta"]), _ptr(out["d_init"]),
+        _ptr(workspace), ws_bytes, _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_backward")
+    return out
 
 
 def prefill_noalloc(q, k, v, log_alpha, beta, cu_seqlens, init_state=None, *,
@@ -188,6 +284,42 @@ def prefill_noalloc(q, k, v, log_alpha, beta, cu_seqlens, init_state=None, *,
     if st != KDA_OK:
         raise KdaError(st, "kda_prefill_noalloc")
     return o, final_state
+
+
+def decode(q, k, v, log_alpha, beta, state, *, gate="channel", raw_qk=False, raw_beta=False,
+           raw_gate=False, o=None, stream=None):
+    """T tokens per sequence (1 <= T <= 16) against the cached ``state``
+    [B, H, dk, dv] fp32, updated in place (one read and one write of it).
+    q, k [B, T, H, dk]; v [B, T, H, dv]; beta [B, T, H]; log_alpha
+    [B, T, H, dk] / [B, T, H] / None per ``gate``. Returns o [B, T, H, dv]."""
+    if gate not in GATES:
+        raise ValueError("gate must be one of %s" % list(GATES))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    code = _dtype_code(q)
+    _check(q, "q", (B, T, H, dk), dt, dev)
+    _check(k, "k", (B, T, H, dk), dt, dev)
+    _check(v, "v", (B, T, H, dv), dt, dev)
+    if gate == "channel":
+        _check(log_alpha, "log_alpha", (B, T, H, dk), torch.float32, dev)
+    elif gate == "scalar":
+        _check(log_alpha, "log_alpha", (B, T, H), torch.float32, dev)
+    else:
+        log_alpha = None
+    _check(beta, "beta", (B, T, H), torch.float32, dev)
+    _check(state, "state", (B, H, dk, dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+    else:
+        _check(o, "o", (B, T, H, dv), dt, dev)
+    st = lib().kda_decode_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                             _ptr(state), int(B), int(T), int(H), int(dk), int(dv), code,
+                             GATES[gate], _flags(raw_qk, raw_beta, raw_gate), _ptr(o),
+                             _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_decode_ex")
+    return o
 
 
 def decode_step(q, k, v, log_alpha, beta, state, *, o=None, stream=None):

@@ -58,6 +58,36 @@ typedef enum {
     KDA_BF16 = 1               /* q, k, v and o are bf16                       */
 } kda_dtype;
 
+/*
+ * Gate forms (the decay alpha that multiplies the state before each token's
+ * read). "22580: from GPT-2 to Kimi K3, explained": "KDA / Kimi Linear" (one
+ * decay per key channel), "Gated Delta Net" (one data-dependent scalar per
+ * token, multiplying the whole previous state), "DeltaNet, or Fast Weight
+ * Programmers" (no decay: the plain delta rule).
+ */
+typedef enum {
+    KDA_GATE_CHANNEL = 0,      /* log_alpha [.., H, dk] fp32                   */
+    KDA_GATE_SCALAR = 1,       /* log_alpha [.., H] fp32, same on every channel */
+    KDA_GATE_NONE = 2          /* alpha = 1; log_alpha unused, may be NULL      */
+} kda_gate;
+
+/*
+ * Input prologue flags: raw projections instead of ready inputs, as the
+ * cached forward of "DeltaNet, or Fast Weight Programmers" computes them just
+ * before the recurrence. Each flag applies its transform inside the kernel:
+ *   KDA_RAW_QK    q and k are raw: each token's head vector x becomes
+ *                 silu(x) / max(|silu(x)|_2, 1e-12)  (F.normalize of SiLU)
+ *   KDA_RAW_BETA  beta holds logits: beta = sigmoid(beta)
+ *   KDA_RAW_GATE  log_alpha holds gate logits x: alpha = sigmoid(x), i.e.
+ *                 log_alpha = log sigmoid(x) (a decay between 0 and 1)
+ */
+#define KDA_RAW_QK   0x1u
+#define KDA_RAW_BETA 0x2u
+#define KDA_RAW_GATE 0x4u
+
+/* Most tokens per sequence one kda_decode_ex call takes. */
+#define KDA_DECODE_MAX_TOKENS 16
+
 /* Lower bound applied to log_alpha by the chunked prefill path. */
 #define KDA_CHUNK_LOG_ALPHA_MIN (-10.0f)
 
@@ -71,11 +101,20 @@ const char *kda_status_string(kda_status status);
 int kda_version(void);
 
 /*
- * Bytes of workspace kda_prefill needs for n_seq packed sequences (the
- * longest-first work order of the variable-length driver). 0 when
- * cu_seqlens will be NULL. Never fails; n_seq < 0 is treated as 0.
+ * Bytes of device workspace kda_prefill needs for a call with these
+ * arguments (the same n_seq, H, dk, dv, dtype and chunk, and whether
+ * cu_seqlens is given). It is non-zero only when the chunked tensor-core
+ * kernel serves the call (bf16, dk = dv = 128, chunk = 64) and then holds:
+ *   - the longest-first order of packed sequences (n_seq int32), when
+ *     cu_seqlens is given;
+ *   - one dk x dv fp32 hand-over slot per (sequence, head) chain, when there
+ *     are at most 128 chains: a ring of CTAs may then serve each chain and
+ *     passes the state between its CTAs through the slot.
+ * Each part starts on a 256-byte boundary. Never fails; negative sizes count
+ * as 0.
  */
-size_t kda_prefill_workspace_bytes(int n_seq, int has_cu_seqlens);
+size_t kda_prefill_workspace_bytes(int n_seq, int H, int dk, int dv, kda_dtype dtype,
+                                   int chunk, int has_cu_seqlens);
 
 /*
  * kda_prefill -- run the recurrence over whole sequences (prefill), with an
@@ -97,15 +136,18 @@ size_t kda_prefill_workspace_bytes(int n_seq, int has_cu_seqlens);
  *   never an out-of-bounds access (each sequence is clamped to [0, T)).
  * chunk: 0 selects the token-recurrent kernel (fp32 state in registers, any
  *   supported head size and dtype, exact gate). 64 selects the chunked
- *   tensor-core kernel (tcgen05 MMAs with TMEM accumulators; bf16 inputs,
- *   dk = dv = 128). With dtype KDA_F32 the recurrent kernel always runs.
+ *   tensor-core kernel (tcgen05 MMAs with TMEM accumulators) for bf16 inputs
+ *   with dk = dv = 128; other dtypes and head sizes run the token-recurrent
+ *   kernel whatever the chunk.
  * final_state may alias init_state (each chain reads its initial state
  *   before writing its final one). o must not alias any input.
  * The chunked kernel needs q, k, v, o, log_alpha and final_state 16-byte
  *   aligned (it moves them in 8- and 16-byte vectors); otherwise
  *   KDA_ERR_INVALID_ARG and nothing is launched.
- * workspace: at least kda_prefill_workspace_bytes(n_seq, cu_seqlens != NULL)
- *   bytes of device memory, 256-byte aligned; may be NULL when that is 0.
+ * workspace: at least kda_prefill_workspace_bytes(n_seq, H, dk, dv, dtype,
+ *   chunk, cu_seqlens != NULL) bytes of device memory, 256-byte aligned, not
+ *   shared with a call that may run at the same time; may be NULL when that
+ *   is 0. Missing or too small: KDA_ERR_WORKSPACE, nothing launched.
  */
 kda_status kda_prefill(const void *q, const void *k, const void *v,
                        const float *log_alpha, const float *beta,
@@ -131,6 +173,86 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v,
                            kda_dtype dtype, void *o, cudaStream_t stream);
 
 /*
+ * kda_prefill_ex -- kda_prefill with a gate form and an input prologue.
+ * Arguments as kda_prefill, plus:
+ *   gate   KDA_GATE_CHANNEL: log_alpha [B, T, H, dk] (kda_prefill's form);
+ *          KDA_GATE_SCALAR:  log_alpha [B, T, H], one decay per token and head
+ *                            (Gated DeltaNet; 4 bytes per head-token read
+ *                            instead of 4 * dk);
+ *          KDA_GATE_NONE:    no decay (DeltaNet); log_alpha may be NULL.
+ *   flags  any of KDA_RAW_QK, KDA_RAW_BETA, KDA_RAW_GATE (see above); 0 for
+ *          ready inputs. With KDA_RAW_GATE the values in log_alpha are logits
+ *          (same shape as the gate form says).
+ * Both kernels take every form; the chunked kernel clamps the resulting
+ * log_alpha at KDA_CHUNK_LOG_ALPHA_MIN as in kda_prefill. Unknown gate or
+ * flag bits: KDA_ERR_INVALID_ARG. kda_prefill is kda_prefill_ex with
+ * KDA_GATE_CHANNEL and flags 0. The workspace is the same as kda_prefill's.
+ */
+kda_status kda_prefill_ex(const void *q, const void *k, const void *v,
+                          const float *log_alpha, const float *beta,
+                          const float *init_state, const int32_t *cu_seqlens,
+                          int n_seq, int B, int T, int H, int dk, int dv,
+                          kda_dtype dtype, kda_gate gate, unsigned flags, int chunk,
+                          void *o, float *final_state,
+                          void *workspace, size_t workspace_bytes,
+                          cudaStream_t stream);
+
+/*
+ * kda_decode_ex -- T tokens per sequence (1 <= T <= KDA_DECODE_MAX_TOKENS)
+ * against a cached state, updated in place: the same result as T successive
+ * kda_decode_step calls (or kda_prefill over the T tokens from that state),
+ * with each head's state read once and written once per call (the
+ * multi-token decode of speculative verification or short appends).
+ *   q, k       [B, T, H, dk]  dtype           v, o  [B, T, H, dv]  dtype
+ *   log_alpha  per `gate`: [B, T, H, dk], [B, T, H] or unused (NULL allowed)
+ *   beta       [B, T, H] fp32                 state [B, H, dk, dv] fp32
+ *   gate, flags as for kda_prefill_ex.
+ * T > KDA_DECODE_MAX_TOKENS: KDA_ERR_UNSUPPORTED (use kda_prefill with
+ * init_state). kda_decode_step is kda_decode_ex with T = 1,
+ * KDA_GATE_CHANNEL and flags 0. The gate is applied exactly (no clamp).
+ */
+kda_status kda_decode_ex(const void *q, const void *k, const void *v,
+                         const float *log_alpha, const float *beta,
+                         float *state, int B, int T, int H, int dk, int dv,
+                         kda_dtype dtype, kda_gate gate, unsigned flags,
+                         void *o, cudaStream_t stream);
+
+/*
+ * kda_backward -- gradients of a loss through the recurrence (the reverse
+ * mode a training step needs; "22580: from GPT-2 to Kimi K3, explained",
+ * section "DeltaNet, or Parallelizing Linear Transformers with Delta Rule",
+ * motivates the chunk-wise form by hardware-efficient training). Given the
+ * forward inputs and dL/do (and optionally dL/dS_final), returns dL/dq,
+ * dL/dk, dL/dv, dL/dlog_alpha, dL/dbeta and dL/dS_0, all fp32:
+ *   q, k, v, log_alpha, beta, init_state, cu_seqlens, n_seq, B, T, H, dk, dv,
+ *   dtype, gate   as for kda_prefill_ex (ready inputs: no prologue flags)
+ *   d_o        [B, T, H, dv] dtype           d_final [n_seq, H, dk, dv] fp32 or NULL
+ *   dq, dk_out [B, T, H, dk] fp32            dv_out  [B, T, H, dv] fp32
+ *   dlog_alpha the gate's shape, fp32 (NULL with KDA_GATE_NONE)
+ *   dbeta      [B, T, H] fp32                d_init  [n_seq, H, dk, dv] fp32 or NULL
+ * The gate is applied exactly (no clamp). Work: a forward pass that stores
+ * the state every 16 tokens in the workspace, then a reverse sweep that
+ * recomputes each 16-token block from its checkpoint (token-recurrent, one
+ * CTA per (sequence, head, 32 value columns)). The column slices of a head
+ * add their parts of dq, dk, dlog_alpha and dbeta with atomic adds, so those
+ * can differ between runs in the last bits. init_state, d_final and d_init
+ * must be 16-byte aligned. workspace: at least
+ * kda_backward_workspace_bytes(n_seq, B * T, H, dk, dv) bytes, 256-byte
+ * aligned (missing or small: KDA_ERR_WORKSPACE).
+ */
+size_t kda_backward_workspace_bytes(int n_seq, int64_t tokens, int H, int dk, int dv);
+
+kda_status kda_backward(const void *q, const void *k, const void *v,
+                        const float *log_alpha, const float *beta,
+                        const float *init_state, const int32_t *cu_seqlens,
+                        int n_seq, int B, int T, int H, int dk, int dv,
+                        kda_dtype dtype, kda_gate gate,
+                        const void *d_o, const float *d_final,
+                        float *dq, float *dk_out, float *dv_out, float *dlog_alpha,
+                        float *dbeta, float *d_init,
+                        void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * kda_prefill_noalloc -- the packed variable-length chunked prefill of
  * kda_prefill (cu_seqlens given, bf16, dk = dv = 128, chunk = 64) for callers
  * that cannot allocate device memory. The source pages have no counterpart:
@@ -152,7 +274,10 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v,
  * overlaps on the GPU race on it; calls on one stream are ordered and safe.
  * The first call on a device looks up the scratch's device address (once per
  * device, with that device current); make that first call before any stream
- * capture begins. Allocates nothing and calls no allocating routine.
+ * capture begins. The address is kept for the life of the process: after a
+ * cudaDeviceReset of that device it is stale, so do not call this entry point
+ * on a device that was reset. Allocates nothing and calls no allocating
+ * routine.
  */
 kda_status kda_prefill_noalloc(const void *q, const void *k, const void *v,
                                const float *log_alpha, const float *beta,

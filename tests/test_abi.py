@@ -39,11 +39,22 @@ def test_status_strings_and_version():
 
 
 def test_workspace_query():
-    assert kda.workspace_bytes(64, False) == 0
-    assert kda.workspace_bytes(0, True) == 0
-    assert kda.workspace_bytes(1, True) == 256
-    assert kda.workspace_bytes(64, True) == 256
-    assert kda.workspace_bytes(65, True) == 512
+    W = lambda n, H, has_cu, dtype=kda.KDA_BF16, chunk=64, d=128: kda.workspace_bytes(
+        n, H, d, d, dtype, chunk, has_cu)
+    slot = 128 * 128 * 4
+    # order of packed sequences: one int32 each, 256-byte granules
+    assert W(1024, 1, True) == 4096
+    assert W(1025, 1, True) == 4096 + 256
+    # few chains (<= 128): one hand-over slot per chain after the order
+    assert W(64, 2, False) == 128 * slot
+    assert W(64, 2, True) == 256 + 128 * slot
+    assert W(1, 1, True) == 256 + slot
+    assert W(129, 1, False) == 0
+    assert W(0, 4, True) == 0
+    # no workspace when the token-recurrent kernel serves the call
+    assert W(4, 2, True, chunk=0) == 0
+    assert W(4, 2, True, dtype=kda.KDA_F32) == 0
+    assert W(4, 2, True, d=64) == 0
 
 
 def _prefill(**kw):
@@ -70,10 +81,12 @@ def _prefill(**kw):
     (dict(dk=96), kda.KDA_ERR_UNSUPPORTED),
     (dict(dv=32), kda.KDA_ERR_UNSUPPORTED),
     (dict(chunk=32), kda.KDA_ERR_UNSUPPORTED),
-    (dict(dk=64, dv=64), kda.KDA_ERR_UNSUPPORTED),        # chunked path is dk = dv = 128
     (dict(cu=FAKE, n_seq=4), kda.KDA_ERR_WORKSPACE),       # varlen needs its workspace
     (dict(cu=FAKE, n_seq=4, ws=FAKE, ws_bytes=16), kda.KDA_ERR_WORKSPACE),
-    (dict(cu=FAKE, n_seq=4, ws=ctypes.c_void_p(0x10004), ws_bytes=256), kda.KDA_ERR_WORKSPACE),
+    (dict(cu=FAKE, n_seq=4, ws=ctypes.c_void_p(0x10004), ws_bytes=1 << 24),
+     kda.KDA_ERR_WORKSPACE),
+    (dict(B=2), kda.KDA_ERR_WORKSPACE),                    # few chains: hand-over slots
+    (dict(B=2, ws=FAKE, ws_bytes=2 * 2 * 65536 - 1), kda.KDA_ERR_WORKSPACE),
     # the chunked kernel moves its tensors in 16-byte vectors
     (dict(la=ctypes.c_void_p(0x10008)), kda.KDA_ERR_INVALID_ARG),
     (dict(k=ctypes.c_void_p(0x10008)), kda.KDA_ERR_INVALID_ARG),
@@ -115,6 +128,9 @@ def test_decode_rejects_bad_arguments(kw, status):
 def test_launch_without_device_reports_cuda_error():
     assert _decode() == kda.KDA_ERR_CUDA
     assert _prefill(chunk=0) == kda.KDA_ERR_CUDA
+    # bf16 with dk = dv = 64 is served by the token-recurrent kernel (no workspace)
+    assert _prefill(dk=64, dv=64) == kda.KDA_ERR_CUDA
+    assert _prefill(B=2, ws=FAKE, ws_bytes=2 * 2 * 65536) == kda.KDA_ERR_CUDA
 
 
 def test_python_wrapper_checks_shapes_before_the_library():

@@ -1,11 +1,14 @@
 """Parity at the full workload sizes, in the launch configuration the
-benchmark times, on outputs the oracle can compute one chain at a time.
+benchmark times.
 
-Workloads: prefill B=4 H=16 T=8192 d=128 (chunk 64); decode B=256 H=32 d=128;
-packed varlen 64 sequences log-uniform in [128, 32768] with H=32; long
-prefill T=1,048,576 H=32 followed by decode steps. The large inputs are
-drawn on the GPU by the seeded generator and the sampled slices are copied to
-the host for the oracle. Tolerances as in test_gpu_parity (normwise).
+Workloads: prefill B=4 H=16 T=8192 d=128 (chunk 64): every chain; decode
+B=256 H=32 d=128 for 1000 in-place steps: every head's output at every step
+and every head's state after the last step; packed varlen 64 sequences
+log-uniform in [128, 32768] with H=32: every sequence on four heads; long
+prefill T=1,048,576 H=32: the first 16384 tokens of every head, the whole
+sequence against a split prefill, then decode steps. The large inputs are
+drawn on the GPU by the seeded generator and copied to the host for the
+oracle. Tolerances as in test_gpu_parity (normwise).
 """
 import numpy as np
 import pytest
@@ -15,63 +18,71 @@ import oracle
 from gated_delta_rule_61_b200 import kda
 from gated_delta_rule_61_b200.inputs import (decode_inputs, decode_state, prefill_inputs,
                                              varlen_lengths)
-from tests.parity import TOL_BF16_O, TOL_BF16_STATE, TOL_F32, assert_close
+from tests.parity import TOL_BF16_O, TOL_BF16_STATE, TOL_F32, assert_close, normwise
 
 pytestmark = pytest.mark.gpu
 CLAMP = kda.CHUNK_LOG_ALPHA_MIN
 
 
-def _chain_oracle(q, k, v, la, b, s0):
-    """One (sequence, head) chain: q, k, la [T, dk]; v [T, dv]; b [T]; s0 [dk, dv]."""
-    o, s = oracle.kda_forward(q[:, None], k[:, None], v[:, None],
-                              la.double().clamp(min=CLAMP)[:, None], b[:, None],
-                              init_state=None if s0 is None else s0[None, None])
-    return o[:, 0], s[0, 0]
-
-
-def test_prefill_mid_full_size_sampled_chains():
+def test_prefill_mid_full_size_every_chain():
     B, T, H, d = 4, 8192, 16, 128
     inp = prefill_inputs(B, T, H, d, d, dtype=torch.bfloat16, seed=0, init_std=0.1,
                          device="cuda")
     o, s = kda.prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
                        init_state=inp["init_state"], chunk=64)
     torch.cuda.synchronize()
-    for b, h in ((0, 0), (1, 7), (3, 15)):
-        sl = lambda x: x[b, :, h].cpu()
-        o_ref, s_ref = _chain_oracle(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]),
-                                     sl(inp["log_alpha"]), inp["beta"][b, :, h].cpu(),
-                                     inp["init_state"][b, h].cpu())
-        assert_close(o[b, :, h], o_ref, TOL_BF16_O, "o chain (%d,%d)" % (b, h))
-        assert_close(s[b, h], s_ref, TOL_BF16_STATE, "state chain (%d,%d)" % (b, h))
+    host = {n: inp[n].cpu() for n in ("q", "k", "v", "log_alpha", "beta", "init_state")}
+    o_ref, s_ref = oracle.kda_forward(host["q"], host["k"], host["v"],
+                                      host["log_alpha"].double().clamp(min=CLAMP),
+                                      host["beta"], init_state=host["init_state"])
+    o_h, s_h = o.cpu(), s.cpu()
+    worst_o = max(normwise(o_h[b, :, h], o_ref[b, :, h]) for b in range(B) for h in range(H))
+    worst_s = max(normwise(s_h[b, h], s_ref[b, h]) for b in range(B) for h in range(H))
+    assert worst_o <= TOL_BF16_O, "o, worst of 64 chains: %.3e" % worst_o
+    assert worst_s <= TOL_BF16_STATE, "final state, worst of 64 chains: %.3e" % worst_s
 
 
-def test_decode_full_size():
-    B, H, d = 256, 32, 128
+def test_decode_full_size_1000_steps():
+    """1000 in-place decode steps at B=256, H=32. The oracle runs each head's
+    1000 steps as one token loop from the same initial state (a decode step is
+    the recurrence with one token), in blocks of heads."""
+    B, H, d, n_steps = 256, 32, 128, 1000
     S = decode_state(B, H, d, d, std=0.05, seed=3, device="cuda")
-    S_host = S.cpu().double().numpy()
-    heads = [(0, 0), (17, 5), (255, 31), (128, 16)]
-    for step in range(4):
+    S0 = S.cpu()
+    names = ("q", "k", "v", "log_alpha", "beta")
+    ins = {n: [] for n in names}
+    outs = torch.empty(n_steps, B, H, d, dtype=torch.bfloat16, device="cuda")
+    for step in range(n_steps):
         inp = decode_inputs(B, H, d, d, dtype=torch.bfloat16, seed=3, step=step, device="cuda")
-        o = kda.decode_step(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], S)
-        torch.cuda.synchronize()
-        if step == 0:   # every head on the first step
-            o_ref, S_host = oracle.kda_decode_step(*(inp[n].cpu() for n in
-                                                     ("q", "k", "v", "log_alpha", "beta")),
-                                                   S_host)
-            assert_close(o, o_ref, TOL_BF16_O, "decode o, all heads")
-            assert_close(S, S_host, TOL_F32, "decode state, all heads")
-        else:           # sampled heads afterwards, continuing from the host copy
-            for b, h in heads:
-                sub = lambda n: inp[n][b:b + 1, h:h + 1].cpu()
-                o_ref, s_new = oracle.kda_decode_step(sub("q"), sub("k"), sub("v"),
-                                                      sub("log_alpha"), sub("beta"),
-                                                      S_host[b:b + 1, h:h + 1])
-                S_host[b:b + 1, h:h + 1] = s_new
-                assert_close(o[b, h], o_ref[0, 0], TOL_BF16_O, "decode o (%d,%d)" % (b, h))
-                assert_close(S[b, h], s_new[0, 0], TOL_F32, "decode state (%d,%d)" % (b, h))
+        kda.decode_step(*(inp[n] for n in names), S, o=outs[step])
+        for n in names:
+            ins[n].append(inp[n])
+    torch.cuda.synchronize()
+    st, detail = kda.device_status()
+    assert st == kda.KDA_OK, (st, detail)
+    # [steps, B * H, d] token-major layout: each head is a chain of 1000 tokens
+    seq = {n: torch.stack(ins[n]).reshape(n_steps, B * H, -1) for n in ("q", "k", "v",
+                                                                      "log_alpha")}
+    seq["beta"] = torch.stack(ins["beta"]).reshape(n_steps, B * H)
+    del ins
+    outs = outs.reshape(n_steps, B * H, d)
+    S_gpu = S.reshape(B * H, d, d).cpu()
+    S0 = S0.reshape(B * H, d, d)
+    worst_o = worst_s = 0.0
+    blk = 512
+    for h0 in range(0, B * H, blk):
+        sl = slice(h0, h0 + blk)
+        o_ref, s_ref = oracle.kda_forward(*(seq[n][:, sl].cpu() for n in names),
+                                          init_state=S0[None, sl])
+        o_blk = outs[:, sl].cpu().double().numpy()
+        for step in range(n_steps):      # every head's output at every step
+            worst_o = max(worst_o, normwise(o_blk[step], o_ref[step]))
+        worst_s = max(worst_s, normwise(S_gpu[sl], s_ref[0]))
+    assert worst_o <= TOL_BF16_O, "decode o, worst step: %.3e" % worst_o
+    assert worst_s <= TOL_F32, "decode state after 1000 steps: %.3e" % worst_s
 
 
-def test_varlen_full_size_sampled_sequences():
+def test_varlen_full_size_every_sequence():
     lengths = varlen_lengths(64, 128, 32768, seed=0)
     H, d = 32, 128
     inp = prefill_inputs(1, 0, H, d, d, dtype=torch.bfloat16, seed=0, init_std=0.1,
@@ -80,22 +91,32 @@ def test_varlen_full_size_sampled_sequences():
                        init_state=inp["init_state"], cu_seqlens=inp["cu_seqlens"], chunk=64)
     torch.cuda.synchronize()
     cu = inp["cu_seqlens"].tolist()
-    order = np.argsort(lengths)
-    picks = [int(order[0]), int(order[len(order) // 2]), int(order[-1])]   # short, mid, longest
-    for i in picks:
-        h = (7 * i) % H
-        a, e = cu[i], cu[i + 1]
-        sl = lambda x: x[0, a:e, h].cpu()
-        o_ref, s_ref = _chain_oracle(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]),
-                                     sl(inp["log_alpha"]), inp["beta"][0, a:e, h].cpu(),
-                                     inp["init_state"][i, h].cpu())
-        assert_close(o[0, a:e, h], o_ref, TOL_BF16_O, "o seq %d (len %d)" % (i, e - a))
-        assert_close(s[i, h], s_ref, TOL_BF16_STATE, "state seq %d (len %d)" % (i, e - a))
+    host = {n: inp[n][0].cpu() for n in ("q", "k", "v", "log_alpha", "beta")}
+    o_h, s_h, s0 = o[0].cpu(), s.cpu(), inp["init_state"].cpu()
+    cu64 = np.asarray(cu, dtype=np.int64)
+    for off in (0, 11, 19, 30):
+        # every sequence on head (7 i + off) mod H, as one packed call of
+        # single-head chains (the oracle threads over them)
+        heads = [(7 * i + off) % H for i in range(len(lengths))]
+        pick = lambda x: torch.cat([x[cu[i]:cu[i + 1], heads[i]:heads[i] + 1]
+                                    for i in range(len(lengths))])
+        o_ref, s_ref = oracle.kda_forward(
+            pick(host["q"]), pick(host["k"]), pick(host["v"]),
+            pick(host["log_alpha"]).double().clamp(min=CLAMP), pick(host["beta"]),
+            init_state=torch.stack([s0[i, h:h + 1] for i, h in enumerate(heads)]),
+            cu_seqlens=cu64)
+        o_gpu = pick(o_h)
+        for i, h in enumerate(heads):
+            a, e = cu[i], cu[i + 1]
+            assert_close(o_gpu[a:e, 0], o_ref[a:e, 0], TOL_BF16_O,
+                         "o seq %d head %d (len %d)" % (i, h, e - a))
+            assert_close(s_h[i, h], s_ref[i, 0], TOL_BF16_STATE,
+                         "state seq %d head %d (len %d)" % (i, h, e - a))
 
 
 def test_long_context_prefill_then_decode():
     """T = 1,048,576, H = 32, zero initial state: the first 16384 tokens of
-    sampled heads against the oracle; the whole sequence against a split
+    every head against the oracle; the whole sequence against a split
     prefill (at 524288 + 37) resumed from the first part's state; then decode
     steps from the final state, checked by the oracle started from the GPU's
     final state."""
@@ -104,11 +125,13 @@ def test_long_context_prefill_then_decode():
     o, s = kda.prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], chunk=64)
     torch.cuda.synchronize()
     n0 = 16384
-    for h in (0, 13, 31):
-        sl = lambda x: x[0, :n0, h].cpu()
-        o_ref, _ = _chain_oracle(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]),
-                                 sl(inp["log_alpha"]), inp["beta"][0, :n0, h].cpu(), None)
-        assert_close(o[0, :n0, h], o_ref, TOL_BF16_O, "o first %d tokens, head %d" % (n0, h))
+    head = {n: inp[n][:, :n0].cpu() for n in ("q", "k", "v", "log_alpha", "beta")}
+    o_ref, _ = oracle.kda_forward(head["q"], head["k"], head["v"],
+                                  head["log_alpha"].double().clamp(min=CLAMP), head["beta"])
+    o_h = o[:, :n0].cpu()
+    for h in range(H):
+        assert_close(o_h[0, :, h], o_ref[0, :, h], TOL_BF16_O,
+                     "o first %d tokens, head %d" % (n0, h))
     part = lambda x, a, e: x[:, a:e].contiguous()
     names = ("q", "k", "v", "log_alpha", "beta")
     o1, s1 = kda.prefill(*(part(inp[n], 0, split) for n in names), chunk=64)

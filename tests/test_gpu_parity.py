@@ -126,6 +126,22 @@ def test_chunk_clamped_gate_is_close_to_a_clear(gate):
     assert_close(s, s_ref, TOL_BF16_STATE, "final state")
 
 
+@pytest.mark.parametrize("B,T,H", [(2, 333, 3), (1, 200, 40), (1, 130, 80)])
+def test_chunk_strong_gates_against_the_unclamped_oracle(B, T, H):
+    """Per-token, per-channel gates drawn uniformly in [-30, 0] straddle the
+    chunked kernel's clamp at -10; its result stays within the bf16
+    tolerances of the EXACT (unclamped) oracle. Shapes cover a ring of two
+    CTAs (6 chains), two CTAs (40 chains) and one CTA per chain (80 chains)."""
+    inp = prefill_inputs(B, T, H, 128, 128, dtype=torch.bfloat16, seed=41 + H, init_std=0.1)
+    g = torch.Generator().manual_seed(1234 + H)
+    inp["log_alpha"] = (-30.0 * torch.rand(inp["log_alpha"].shape, generator=g,
+                                           dtype=torch.float64)).float()
+    o_ref, s_ref = _oracle(inp)            # no clamp
+    o, s = _gpu_prefill(inp, 64)
+    assert_close(o, o_ref, TOL_BF16_O, "o vs unclamped oracle")
+    assert_close(s, s_ref, TOL_BF16_STATE, "final state vs unclamped oracle")
+
+
 @pytest.mark.parametrize("gate", [-5.0, -60.0, -np.inf])
 def test_recurrent_applies_the_gate_exactly(gate):
     inp = prefill_inputs(1, 40, 2, 128, 128, dtype=torch.float32, seed=22, init_std=1.0)
