@@ -95,21 +95,11 @@ constexpr uint32_t MISC_GAMMA = 0, MISC_BETA = 512, MISC_PAIR = 1280,
                    MISC_GF = 17664, MISC_GL = 19712, MISC_MBAR = 21760, MISC_FULL = 21776,
                    MISC_TMEM = 21784, MISC_TOT4 = 21792,
                    MISC_NORM = 23840,   // raw q/k: per-warp partial squared norms [16][16]
-                   MISC_BARA = 24864, MISC_BARB = 24872,   // input-copy mbarriers
-                   MISC_SGATE = 24896;  // scalar gate: one log-decay per row [64]
-constexpr uint32_t kSmemBytes = OFF_MISC + 25152 + 1024;
-// Landing places of the next own chunk's raw inputs (tensor-map copies, 128B
-// swizzled [row][channel] tiles like the operand tiles): k lands in the
-// K e^g tile and q in the Q e^g tile (P1 rewrites both in place), v in its
-// MMA operand tile directly, and log_alpha (four 32-channel boxes of 8 KiB)
-// in the parts of the Gram tiles that are dead from the W/U MMA on (T tile
-// and the tail of A; the solve's scratch in B). k, v and log_alpha are copied
-// as soon as the W/U MMA has read the previous contents, q once the D/O MMA
-// has.
-__device__ __forceinline__ uint32_t lambda_box(int b) {
-  return b == 0 ? OFF_AG + 16384 : b == 1 ? OFF_AG + 24576 : b == 2 ? OFF_BG + 16384
-                                                                     : OFF_BG + 24576;
-}
+                   MISC_BARA = 24864;   // mbarrier of the k/v tensor-map copies
+constexpr uint32_t kSmemBytes = OFF_MISC + 24880 + 1024;
+// The next own chunk's raw k and v land by tensor-map copies (128B-swizzled
+// [row][channel] tiles, the operand tiles' layout): k in the K e^g tile (P1
+// rewrites it in place) and v directly in its MMA operand tile.
 // State hand-over between the CTAs of a chain's cluster goes through the
 // chain's hand-over slot in global memory (64 KiB, L2-resident; a workspace
 // region, or the chain's own final_state): it is
@@ -195,6 +185,25 @@ __device__ __forceinline__ bool cta_wait(uint32_t mbar, uint32_t parity, int cod
   tc::fence_after_sync();
   if (fail && threadIdx.x == 0) report_timeout(code);
   return fail == 0;
+}
+
+// Same, for two barriers: the MMA barrier and, when need2, the input-copy
+// barrier of the next own chunk (waited here so that chunk's P1 needs no
+// barrier of its own). Returns 0, or 1 / 2 for the wait that gave up.
+__device__ __forceinline__ int cta_wait2(uint32_t mbar, uint32_t parity, uint32_t mbar2,
+                                         uint32_t parity2, bool need2, int code) {
+  int fail = 0;
+  if (threadIdx.x == 0) {
+    fail = tc::mbar_wait_bounded(mbar, parity, kMaxWaitNs) ? 0 : 1;
+    if (!fail && need2) fail = tc::mbar_wait_bounded(mbar2, parity2, kMaxWaitNs) ? 0 : 2;
+  }
+  const int any = __syncthreads_or(fail);
+  tc::fence_after_sync();
+  if (!any) return 0;
+  // (failure path only: tell every thread which wait gave up)
+  const int first = __syncthreads_or(fail == 1);
+  if (threadIdx.x == 0) report_timeout(code);
+  return first ? 1 : 2;
 }
 
 __device__ __forceinline__ void cta_sync_tc() {
@@ -388,9 +397,8 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
                const float* __restrict__ beta, const float* init_state,
                const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ order,
                int T, int H, __nv_bfloat16* __restrict__ o, float* final_state, float* xfer,
-               unsigned flags, const __grid_constant__ CUtensorMap tm_q,
-               const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-               const __grid_constant__ CUtensorMap tm_la) {
+               unsigned flags, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -417,22 +425,20 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     tc::tmem_relinquish();
   }
   const uint32_t mbar_full = sbase + OFF_MISC + MISC_FULL;     // partner's state is in L2
-  const uint32_t bar_a = sbase + OFF_MISC + MISC_BARA;   // k, v, log_alpha landed
-  const uint32_t bar_b = sbase + OFF_MISC + MISC_BARB;   // q landed
+  const uint32_t bar_a = sbase + OFF_MISC + MISC_BARA;   // k and v landed
   if (tid == 0) {
     tc::mbar_init(mbar, 1);
     tc::mbar_init(bar_a, 1);
-    tc::mbar_init(bar_b, 1);
     if (kPair) tc::mbar_init(mbar_full, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   cta_sync_tc();
   if (kPair) tc::cluster_sync();   // partner's barriers exist before any remote arrive
   const uint32_t tmem = *tmem_slot;
-  uint32_t phase = 0, full_phase = 0, phase_a = 0, phase_b = 0;
+  uint32_t phase = 0, full_phase = 0, phase_a = 0;
   // Thread 0 issues the MMAs and the input copies; on a failed wait it lets
   // whatever it issued finish (bounded) before memory is released.
-  bool pend_mma = false, pend_a = false, pend_b = false;
+  bool pend_mma = false, pend_a = false;
   bool ok = true;
 
   const int quad = warp & 3, grp = warp >> 2;
@@ -464,61 +470,60 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
   const int pr = tid & 63, rg = tid >> 6, c0 = 2 * pr;
   float* s_pair = reinterpret_cast<float*>(smem + OFF_MISC + MISC_PAIR);   // [32][128]
   float* s_tot4 = reinterpret_cast<float*>(smem + OFF_MISC + MISC_TOT4);   // [4][128]
-  // Inputs of a chunk. One thread issues the tensor-map copies of k, v and
-  // log_alpha (bar_a) and of q (bar_b); beta (and a scalar gate) are small
-  // and read with plain loads into registers / shared memory.
+  // Inputs of a chunk. k and v arrive by tensor-map copies (one thread,
+  // bar_a) into their operand tiles; they are issued once the W/U MMA has
+  // read those tiles, a whole D/O + update phase before the next own chunk
+  // needs them. log_alpha, q and beta are consumed earlier (the gate scan
+  // runs during the D/O MMA) and have no free landing place that early, so
+  // they are read into registers one own chunk ahead, during the Gram MMA.
+  float2 lr[8];
+  uint32_t qr[8];
   float bt[2];   // warp 0 only: beta of rows 2 lane, 2 lane + 1
-  float* s_sgate = reinterpret_cast<float*>(smem + OFF_MISC + MISC_SGATE);
   auto chunk_len = [&](int nn) {
     const long long tc0 = t_begin + (long long)nn * C;
     return (int)((t_end - tc0) < C ? (t_end - tc0) : C);
   };
-  auto issue_kvl = [&](int nn) {
+  auto issue_kv = [&](int nn) {
     const int z = (int)(t_begin + (long long)nn * C);
-    const int Lc = chunk_len(nn);
     if (tid == 0) {
-      constexpr uint32_t bytes = 2 * 16384u + (kGate == 0 ? 32768u : 0u);
-      tc::mbar_arrive_expect_tx(bar_a, bytes);
+      tc::mbar_arrive_expect_tx(bar_a, 2 * 16384u);
       pend_a = true;
       tc::tma_load_3d(sbase + OFF_BK, &tm_k, 0, head, z, bar_a);
       tc::tma_load_3d(sbase + OFF_BK + 8192, &tm_k, 64, head, z, bar_a);
       tc::tma_load_3d(sbase + OFF_VV, &tm_v, 0, head, z, bar_a);
       tc::tma_load_3d(sbase + OFF_VV + 8192, &tm_v, 64, head, z, bar_a);
-      if constexpr (kGate == 0) {
+    }
+  };
+  auto load_rows = [&](int nn) {
+    const long long tc0 = t_begin + (long long)nn * C;
+    const int Lc = chunk_len(nn);
 #pragma unroll
-        for (int bx = 0; bx < 4; ++bx)
-          tc::tma_load_3d(sbase + lambda_box(bx), &tm_la, 32 * bx, head, z, bar_a);
+    for (int i = 0; i < 8; ++i) {
+      const int r = 16 * (i >> 1) + 2 * rg + (i & 1);
+      lr[i] = make_float2(0.f, 0.f);
+      qr[i] = 0u;
+      if (r < Lc) {
+        const size_t tok = (size_t)(tc0 + r) * H + head;
+        if constexpr (kGate == 0) {
+          lr[i] = ld_stream_f2(log_alpha + tok * DK + c0);
+        } else if constexpr (kGate == 1) {
+          const float x = __ldg(log_alpha + tok);
+          lr[i] = make_float2(x, x);
+        }
+        qr[i] = ld_stream_u32(q + tok * DK + c0);
       }
     }
     bt[0] = bt[1] = 0.f;
     if (warp == 0) {
-      if (2 * lane < Lc) bt[0] = __ldg(beta + (size_t)(z + 2 * lane) * H + head);
-      if (2 * lane + 1 < Lc) bt[1] = __ldg(beta + (size_t)(z + 2 * lane + 1) * H + head);
-    }
-    if constexpr (kGate == 1) {
-      if (warp == 1) {
-        s_sgate[2 * lane] = 2 * lane < Lc ? __ldg(log_alpha + (size_t)(z + 2 * lane) * H + head)
-                                          : 0.f;
-        s_sgate[2 * lane + 1] =
-            2 * lane + 1 < Lc ? __ldg(log_alpha + (size_t)(z + 2 * lane + 1) * H + head) : 0.f;
-      }
-    }
-  };
-  auto issue_q = [&](int nn) {
-    const int z = (int)(t_begin + (long long)nn * C);
-    if (tid == 0) {
-      tc::mbar_arrive_expect_tx(bar_b, 16384u);
-      pend_b = true;
-      tc::tma_load_3d(sbase + OFF_QT, &tm_q, 0, head, z, bar_b);
-      tc::tma_load_3d(sbase + OFF_QT + 8192, &tm_q, 64, head, z, bar_b);
+      if (2 * lane < Lc) bt[0] = __ldg(beta + (size_t)(tc0 + 2 * lane) * H + head);
+      if (2 * lane + 1 < Lc) bt[1] = __ldg(beta + (size_t)(tc0 + 2 * lane + 1) * H + head);
     }
   };
   if (rank < n_chunks) {
-    issue_kvl(rank);
-    issue_q(rank);
-    __syncthreads();   // the scalar gate row is in shared memory
+    issue_kv(rank);
+    load_rows(rank);
   }
-  // Cumulative gates of a chunk from its landed log_alpha tile (after bar_a):
+  // Cumulative gates of a chunk from its log_alpha rows (lr):
   // pair sums per (sub-chunk, rg) -> one exclusive scan over the 32 pairs per
   // channel -> each thread adds its own rows. Writes g0/g1 (registers), beta,
   // the first and last g of every sub-chunk and the chunk's decay e^{g_last}
@@ -527,28 +532,15 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
   float g0[8], g1[8];
   auto gates = [&](int Lc) -> bool {
     {
-      if (!cta_wait(bar_a, phase_a, 6)) return false;
-      phase_a ^= 1;
-      pend_a = false;
       float l0[8], l1[8];
       const bool raw_gate = kGate != 2 && (flags & 4u);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int r = 16 * (i >> 1) + 2 * rg + (i & 1);
-        float x0 = 0.f, x1 = 0.f;   // rows past the chunk's end: no decay
-        if (r < Lc) {
-          if constexpr (kGate == 0) {
-            const float2 lv = *reinterpret_cast<const float2*>(
-                smem + lambda_box(c0 >> 5) + tc::sw128<4>(r, c0 & 31, 64));
-            x0 = lv.x;
-            x1 = lv.y;
-          } else if constexpr (kGate == 1) {
-            x0 = x1 = s_sgate[r];
-          }
-          if (raw_gate) {
-            x0 = log_sigmoid_fast(x0);
-            x1 = kGate == 1 ? x0 : log_sigmoid_fast(x1);
-          }
+        float x0 = lr[i].x, x1 = lr[i].y;   // zero past the chunk's end: no decay
+        if (raw_gate && r < Lc) {
+          x0 = log_sigmoid_fast(x0);
+          x1 = kGate == 1 ? x0 : log_sigmoid_fast(x1);
         }
         l0[i] = fmaxf(x0, kLogAlphaMin);
         l1[i] = fmaxf(x1, kLogAlphaMin);
@@ -640,10 +632,12 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       ok = gates(L);
       if (!ok) break;
     }
-    ok = cta_wait(bar_b, phase_b, 7);   // q of this chunk has landed
-    if (!ok) break;
-    phase_b ^= 1;
-    pend_b = false;
+    if (n == rank) {   // later chunks waited for their k and v at the previous P8
+      ok = cta_wait(bar_a, phase_a, 7);
+      if (!ok) break;
+      phase_a ^= 1;
+      pend_a = false;
+    }
     if constexpr (kRawQK) {
       // Squared norms of SiLU(k) and SiLU(q) per row: this thread's two
       // channels, reduced over the warp's 32 lanes by halving exchanges
@@ -654,11 +648,11 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       float nv[16];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const uint32_t kr = raw_pair(OFF_BK, i), qr = raw_pair(OFF_QT, i);
+        const uint32_t kr = raw_pair(OFF_BK, i);
         const float k0 = silu_tanh(__uint_as_float(kr << 16));
         const float k1 = silu_tanh(__uint_as_float(kr & 0xffff0000u));
-        const float q0 = silu_tanh(__uint_as_float(qr << 16));
-        const float q1 = silu_tanh(__uint_as_float(qr & 0xffff0000u));
+        const float q0 = silu_tanh(__uint_as_float(qr[i] << 16));
+        const float q1 = silu_tanh(__uint_as_float(qr[i] & 0xffff0000u));
         nv[i] = fmaf(k0, k0, k1 * k1);
         nv[8 + i] = fmaf(q0, q0, q1 * q1);
       }
@@ -734,10 +728,12 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       for (int i = 0; i < 8; ++i) {
         const int a = i >> 1, e = i & 1;
         const uint32_t ro = (uint32_t)(a * 2048 + e * 128) + (e ? xo1 : xo0);
-        // bf16 pairs widen exactly: low half << 16, high half masked.
-        const uint32_t kr = raw_pair(OFF_BK, i), qr = raw_pair(OFF_QT, i);
+        // bf16 pairs widen exactly: low half << 16, high half masked. Raw k
+        // is read where K e^g is written (zero past the chunk's end).
+        const uint32_t kr = 16 * a + 2 * rg + e < L ? *reinterpret_cast<const uint32_t*>(pBK + ro)
+                                                    : 0u;
         float k0 = __uint_as_float(kr << 16), k1 = __uint_as_float(kr & 0xffff0000u);
-        float q0 = __uint_as_float(qr << 16), q1 = __uint_as_float(qr & 0xffff0000u);
+        float q0 = __uint_as_float(qr[i] << 16), q1 = __uint_as_float(qr[i] & 0xffff0000u);
         if constexpr (kRawQK) {
           // normalize(silu(x)): divide by max(|silu(x)|, 1e-12) of the row,
           // whose squared norm is the sum of the row group's two warps.
@@ -815,8 +811,10 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       tc::mma_commit(mbar);
       pend_mma = true;
     }
-    // While the Gram MMA runs: warm L2 with the inputs of the own chunk after
-    // next (the next one's are copied in from P5 on).
+    // While the Gram MMA runs: read the next own chunk's log_alpha, q and beta
+    // into registers (this chunk's were consumed by the gate scan and the
+    // tiles) and warm L2 with the inputs of the own chunk after it.
+    if (n + step < n_chunks) load_rows(n + step);
     if (n + 2 * step < n_chunks) {
       const long long t1 = t0 + (long long)(2 * step) * C;
       const int row = tid >> 3, part = tid & 7;
@@ -917,7 +915,9 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       const float* N = reinterpret_cast<const float*>(smem + OFF_NMAT);
       float* X = reinterpret_cast<float*>(smem + OFF_XMAT);
       // Meanwhile warps 8..15 move the previous chunk's output to HBM (staged
-      // in the S0 bf16 tile, which is dead until P5).
+      // in the S0 bf16 tile, which is dead until P5). (Also copying and
+      // decaying the state there, to shorten P5, was measured slower: it
+      // delays the solve's first barrier more than it saves.)
       if (n >= step && warp >= 8)
         store_output_8w(tmem, lane_off, (warp >> 2) & 1, m, smem + OFF_SB, o,
                         t0 - (long long)step * C, C, H, head);
@@ -1002,9 +1002,8 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     if (!ok) break;
     pend_mma = false;
     phase ^= 1;
-    // The W/U MMA has read K e^g, V and T: bring in the next own chunk's k,
-    // v and log_alpha (and its beta / scalar gate).
-    if (n + step < n_chunks) issue_kvl(n + step);
+    // The W/U MMA has read K e^g and V: bring in the next own chunk's k and v.
+    if (n + step < n_chunks) issue_kv(n + step);
     {
       // -W^T to shared memory: lane c holds W^T[c][r]; this warp takes r in [16 grp, +16).
       float w[16];
@@ -1082,7 +1081,6 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     if (!ok) break;
     pend_mma = false;
     phase ^= 1;
-    if (n + step < n_chunks) issue_q(n + step);   // the O MMA has read Q e^g
 
     // ---- P8: S^T += D^T K~ (tf32, A from TMEM, B K-major); O^T += D^T M_qk^T
     if (tid == 0) {
@@ -1101,10 +1099,20 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       tc::mma_commit(mbar);
       pend_mma = true;
     }
-    ok = cta_wait(mbar, phase, 4);
-    if (!ok) break;
-    pend_mma = false;
-    phase ^= 1;
+    {
+      const bool next = n + step < n_chunks;   // its k and v were issued at P5
+      const int f = cta_wait2(mbar, phase, bar_a, phase_a, next, 4);
+      if (f != 1) {
+        pend_mma = false;
+        phase ^= 1;
+      }
+      if (f == 0 && next) {
+        pend_a = false;
+        phase_a ^= 1;
+      }
+      ok = f == 0;
+      if (!ok) break;
+    }
 
     if (kPair && n + 1 < n_chunks) {
       // Hand the state to the next CTA of the ring, which takes chunk n + 1.
@@ -1148,7 +1156,6 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     // released.
     if (pend_mma) tc::mbar_wait_bounded(mbar, phase, kMaxWaitNs);
     if (pend_a) tc::mbar_wait_bounded(bar_a, phase_a, kMaxWaitNs);
-    if (pend_b) tc::mbar_wait_bounded(bar_b, phase_b, kMaxWaitNs);
   }
   cta_sync_tc();
   if (kPair) tc::cluster_sync();   // no remote traffic targets this CTA past this point
@@ -1232,7 +1239,7 @@ struct ChunkArgs {
   __nv_bfloat16* o;
   float *sT, *xfer;
   unsigned flags;
-  CUtensorMap tm_q, tm_k, tm_v, tm_la;
+  CUtensorMap tm_k, tm_v;
 };
 
 // cuTensorMapEncodeTiled, reached through the runtime's driver entry point
@@ -1290,14 +1297,14 @@ static cudaError_t launch_variant(const ChunkArgs& a, long long chains, int ring
     if (ring == 4)
       return cudaLaunchKernelEx(&cfg, chunk64_kernel<4, kGate, kRaw>, a.q, a.k, a.v, a.la,
                                 a.beta, a.s0, a.cu, a.order, a.T, a.H, a.o, a.sT, a.xfer,
-                                a.flags, a.tm_q, a.tm_k, a.tm_v, a.tm_la);
+                                a.flags, a.tm_k, a.tm_v);
     return cudaLaunchKernelEx(&cfg, chunk64_kernel<2, kGate, kRaw>, a.q, a.k, a.v, a.la,
                               a.beta, a.s0, a.cu, a.order, a.T, a.H, a.o, a.sT, a.xfer,
-                              a.flags, a.tm_q, a.tm_k, a.tm_v, a.tm_la);
+                              a.flags, a.tm_k, a.tm_v);
   }
   chunk64_kernel<1, kGate, kRaw><<<(unsigned)chains, kThreads, kSmemBytes, stream>>>(
       a.q, a.k, a.v, a.la, a.beta, a.s0, a.cu, a.order, a.T, a.H, a.o, a.sT, nullptr, a.flags,
-      a.tm_q, a.tm_k, a.tm_v, a.tm_la);
+      a.tm_k, a.tm_v);
   return cudaGetLastError();
 }
 
@@ -1342,25 +1349,19 @@ cudaError_t launch_chunk64(const void* q, const void* k, const void* v, const fl
   a.sT = sT;
   a.xfer = xfer;
   a.flags = flags;
-  // Tensor maps of the token-major inputs: every token of the call (packed:
-  // T; dense batch: n_seq x T).
+  // Tensor maps of k and v over every token of the call (packed: T; dense
+  // batch: n_seq x T).
   PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
   cudaError_t e1 = tensor_map_encoder(&enc);
   if (e1 != cudaSuccess) return e1;
   const long long tokens = cu ? (long long)T : (long long)n_seq * T;
   if (tokens == 0) {
-    memset(&a.tm_q, 0, sizeof(CUtensorMap));   // no chunk to load: never read
-    a.tm_k = a.tm_v = a.tm_la = a.tm_q;
+    memset(&a.tm_k, 0, sizeof(CUtensorMap));   // no chunk to load: never read
+    a.tm_v = a.tm_k;
     return launch_variant<2, false>(a, chains, 1, stream);   // initial -> final states
   }
-  if ((e1 = encode_rows(enc, &a.tm_q, q, true, tokens, H)) != cudaSuccess) return e1;
   if ((e1 = encode_rows(enc, &a.tm_k, k, true, tokens, H)) != cudaSuccess) return e1;
   if ((e1 = encode_rows(enc, &a.tm_v, v, true, tokens, H)) != cudaSuccess) return e1;
-  if (gate == 0) {
-    if ((e1 = encode_rows(enc, &a.tm_la, la, false, tokens, H)) != cudaSuccess) return e1;
-  } else {
-    a.tm_la = a.tm_k;   // not read
-  }
   // Few chains: R = 4 or 2 CTAs per chain (chunks round-robin), all in one
   // wave; the state passes between them through the chain's xfer slot.
   const int ring = (xfer && 2 * chains <= n_sm) ? (4 * chains <= n_sm ? 4 : 2) : 1;

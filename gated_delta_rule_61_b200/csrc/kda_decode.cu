@@ -19,7 +19,8 @@
 // own v entries); 256 threads = 8 warps; every lane streams 128-bit vectors of
 // whole contiguous rows, holds its rows in registers for the whole call, and
 // the two column reductions go through shuffles and one small shared-memory
-// exchange per token.
+// exchange per token. Two kernels: the plain decode step, and the general one
+// (several tokens, gate forms, prologue).
 #include "kda_common.cuh"
 
 namespace kda {
@@ -37,16 +38,18 @@ __device__ __forceinline__ float decay_from(float g, unsigned flags) {
   return (flags & kRawGate) ? sigmoid_f(g) : expf(g);
 }
 
+// The plain decode step (one token, per-channel gate, ready inputs).
 // CTA (head, slice) owns value columns [slice * DV / SPLIT, +DV / SPLIT).
 // Within a CTA each lane owns one 4-column group; LPR = columns / 4 lanes
 // cover a row, so a warp instruction reads RPI = 32 / LPR whole rows (512
-// contiguous bytes per warp for 128 columns).
+// contiguous bytes per warp for 128 columns). 64 registers per thread keep
+// 2 * SPLIT CTAs per SM in flight.
 template <typename TIn, int DK, int DV, int SPLIT>
 __global__ void __launch_bounds__(256, 2 * SPLIT)
-decode_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
-              const float* __restrict__ log_alpha, const float* __restrict__ beta,
-              float* __restrict__ state, TIn* __restrict__ o, int T, int H, int gate,
-              unsigned flags) {
+decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
+                   const TIn* __restrict__ v, const float* __restrict__ log_alpha,
+                   const float* __restrict__ beta, float* __restrict__ state,
+                   TIn* __restrict__ o) {
   constexpr int kWarps = 8;
   constexpr int CW = DV / SPLIT;          // value columns of this CTA
   constexpr int LPR = CW / 4;             // lanes per row (one float4 each)
@@ -54,16 +57,14 @@ decode_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* _
   constexpr int NI = DK / (kWarps * RPI); // float4 per thread
   static_assert(CW % 4 == 0 && 32 % LPR == 0 && DK % (kWarps * RPI) == 0, "shape");
 
-  const int head = blockIdx.x / SPLIT, slice = blockIdx.x % SPLIT;   // head = b * H + h
-  const int b = head / H, h = head - (head / H) * H;
+  const int head = blockIdx.x / SPLIT, slice = blockIdx.x % SPLIT;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cg = lane % LPR, sub = lane / LPR;
   const int col = slice * CW + 4 * cg;
-  const bool raw_qk = flags & kRawQK;
 
-  __shared__ float s_k[2][DK], s_q[2][DK], s_a[2][DK];
-  __shared__ float4 s_red[2][kWarps][2][LPR];
-  __shared__ float s_sum[2][kWarps][3];   // k.q and, for raw inputs, |k|^2 and |q|^2
+  __shared__ float s_k[DK], s_q[DK], s_a[DK];
+  __shared__ float4 s_red[kWarps][2][LPR];
+  __shared__ float s_kq[kWarps];
 
   float* S = state + (size_t)head * DK * DV;
 
@@ -75,45 +76,166 @@ decode_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* _
     s[i] = __ldcs(reinterpret_cast<const float4*>(S + (size_t)row * DV + col));
   }
 
-  for (int t = 0; t < T; ++t) {
-    const int buf = t & 1;
-    const size_t tok = ((size_t)b * T + t) * H + h;      // token index in [B, T, H]
-    // Per-token vectors: k, q (after the prologue when raw), alpha per key row.
-    float part[3] = {0.f, 0.f, 0.f};
-    for (int i = threadIdx.x; i < DK; i += blockDim.x) {
+  // Small per-head vectors: k, q, alpha = exp(log_alpha); k . q per warp.
+  float kq_part = 0.f;
+  for (int i = threadIdx.x; i < DK; i += blockDim.x) {
+    const float kk = Io<TIn>::load(k + (size_t)head * DK + i);
+    const float qq = Io<TIn>::load(q + (size_t)head * DK + i);
+    s_k[i] = kk;
+    s_q[i] = qq;
+    s_a[i] = expf(__ldg(log_alpha + (size_t)head * DK + i));
+    kq_part += kk * qq;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) kq_part += __shfl_xor_sync(0xffffffffu, kq_part, off);
+  if (lane == 0) s_kq[warp] = kq_part;
+  __syncthreads();
+
+  // Decay rows and accumulate partial r = S'^T k and p = S'^T q.
+  float4 r = make_float4(0.f, 0.f, 0.f, 0.f), p = r;
+#pragma unroll
+  for (int i = 0; i < NI; ++i) {
+    const int row = (warp + i * kWarps) * RPI + sub;
+    const float a = s_a[row], kk = s_k[row], qq = s_q[row];
+    s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
+    r.x = fmaf(s[i].x, kk, r.x); r.y = fmaf(s[i].y, kk, r.y);
+    r.z = fmaf(s[i].z, kk, r.z); r.w = fmaf(s[i].w, kk, r.w);
+    p.x = fmaf(s[i].x, qq, p.x); p.y = fmaf(s[i].y, qq, p.y);
+    p.z = fmaf(s[i].z, qq, p.z); p.w = fmaf(s[i].w, qq, p.w);
+  }
+#pragma unroll
+  for (int off = LPR; off < 32; off <<= 1) {   // lanes holding the same columns
+    r.x += __shfl_xor_sync(0xffffffffu, r.x, off); r.y += __shfl_xor_sync(0xffffffffu, r.y, off);
+    r.z += __shfl_xor_sync(0xffffffffu, r.z, off); r.w += __shfl_xor_sync(0xffffffffu, r.w, off);
+    p.x += __shfl_xor_sync(0xffffffffu, p.x, off); p.y += __shfl_xor_sync(0xffffffffu, p.y, off);
+    p.z += __shfl_xor_sync(0xffffffffu, p.z, off); p.w += __shfl_xor_sync(0xffffffffu, p.w, off);
+  }
+  if (sub == 0) {
+    s_red[warp][0][cg] = r;
+    s_red[warp][1][cg] = p;
+  }
+  __syncthreads();
+
+  float kq = 0.f;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) kq += s_kq[w];
+  r = make_float4(0.f, 0.f, 0.f, 0.f);
+  p = r;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const float4 a = s_red[w][0][cg], b = s_red[w][1][cg];
+    r.x += a.x; r.y += a.y; r.z += a.z; r.w += a.w;
+    p.x += b.x; p.y += b.y; p.z += b.z; p.w += b.w;
+  }
+  const float bb = __ldg(beta + head);
+  const float rr[4] = {r.x, r.y, r.z, r.w}, pp[4] = {p.x, p.y, p.z, p.w};
+  float d[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    d[j] = bb * (Io<TIn>::load(v + (size_t)head * DV + col + j) - rr[j]);
+    if (warp == 0 && sub == 0)
+      Io<TIn>::store(o + (size_t)head * DV + col + j, fmaf(kq, d[j], pp[j]));
+  }
+
+  // S = S' + k d^T, written once.
+#pragma unroll
+  for (int i = 0; i < NI; ++i) {
+    const int row = (warp + i * kWarps) * RPI + sub;
+    const float kk = s_k[row];
+    s[i].x = fmaf(kk, d[0], s[i].x); s[i].y = fmaf(kk, d[1], s[i].y);
+    s[i].z = fmaf(kk, d[2], s[i].z); s[i].w = fmaf(kk, d[3], s[i].w);
+    __stcs(reinterpret_cast<float4*>(S + (size_t)row * DV + col), s[i]);
+  }
+}
+
+// Every other decode call (1 to 16 tokens, any gate form, prologue flags):
+// the same state pass, with all T tokens' inputs staged into shared memory
+// first (k, q and the decay per key row after the prologue; v of this CTA's
+// columns; beta, k.q and the normalisation scales per token), which also
+// overlaps those loads with the state loads. The token loop then needs one
+// CTA barrier per token (the cross-warp part of r and p, double-buffered).
+template <typename TIn, int DK, int DV, int SPLIT>
+__global__ void __launch_bounds__(256, 2 * SPLIT)
+decode_multi_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
+                    const TIn* __restrict__ v, const float* __restrict__ log_alpha,
+                    const float* __restrict__ beta, float* __restrict__ state,
+                    TIn* __restrict__ o, int T, int H, int gate, unsigned flags) {
+  constexpr int kWarps = 8, kMaxT = 16;
+  constexpr int CW = DV / SPLIT;
+  constexpr int LPR = CW / 4;
+  constexpr int RPI = 32 / LPR;
+  constexpr int NI = DK / (kWarps * RPI);
+  static_assert(CW % 4 == 0 && 32 % LPR == 0 && DK % (kWarps * RPI) == 0, "shape");
+
+  const int head = blockIdx.x / SPLIT, slice = blockIdx.x % SPLIT;   // head = b * H + h
+  const int b = head / H, h = head - b * H;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cg = lane % LPR, sub = lane / LPR;
+  const int col = slice * CW + 4 * cg;
+  const bool raw_qk = flags & kRawQK;
+
+  __shared__ float s_k[kMaxT][DK], s_q[kMaxT][DK], s_a[kMaxT][DK];
+  __shared__ __align__(16) float s_v[kMaxT][CW];
+  __shared__ float s_beta[kMaxT], s_kq[kMaxT], s_ik[kMaxT], s_iq[kMaxT];
+  __shared__ float4 s_red[2][kWarps][2][LPR];
+
+  float* S = state + (size_t)head * DK * DV;
+  float4 s[NI];
+#pragma unroll
+  for (int i = 0; i < NI; ++i) {
+    const int row = (warp + i * kWarps) * RPI + sub;
+    s[i] = __ldcs(reinterpret_cast<const float4*>(S + (size_t)row * DV + col));
+  }
+
+  // Stage the tokens: warp w takes tokens w, w + 8.
+  for (int t = warp; t < T; t += kWarps) {
+    const size_t tok = ((size_t)b * T + t) * H + h;
+    float kq = 0.f, nk = 0.f, nq = 0.f;
+    for (int i = lane; i < DK; i += 32) {
       float kk = Io<TIn>::load(k + tok * DK + i);
       float qq = Io<TIn>::load(q + tok * DK + i);
       if (raw_qk) {
         kk = silu_f(kk);
         qq = silu_f(qq);
-        part[1] += kk * kk;
-        part[2] += qq * qq;
+        nk = fmaf(kk, kk, nk);
+        nq = fmaf(qq, qq, nq);
       }
-      s_k[buf][i] = kk;
-      s_q[buf][i] = qq;
+      s_k[t][i] = kk;
+      s_q[t][i] = qq;
       float a = 1.f;
       if (gate == kGateChannel) a = decay_from(__ldg(log_alpha + tok * DK + i), flags);
       else if (gate == kGateScalar) a = decay_from(__ldg(log_alpha + tok), flags);
-      s_a[buf][i] = a;
-      part[0] += kk * qq;
+      s_a[t][i] = a;
+      kq = fmaf(kk, qq, kq);
     }
+    for (int j = lane; j < CW; j += 32) s_v[t][j] = Io<TIn>::load(v + tok * DV + slice * CW + j);
 #pragma unroll
-    for (int j = 0; j < 3; ++j)
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) part[j] += __shfl_xor_sync(0xffffffffu, part[j], off);
+    for (int off = 16; off > 0; off >>= 1) {
+      kq += __shfl_xor_sync(0xffffffffu, kq, off);
+      nk += __shfl_xor_sync(0xffffffffu, nk, off);
+      nq += __shfl_xor_sync(0xffffffffu, nq, off);
+    }
     if (lane == 0) {
-      s_sum[buf][warp][0] = part[0];
-      s_sum[buf][warp][1] = part[1];
-      s_sum[buf][warp][2] = part[2];
+      // L2 normalisation of SiLU(k), SiLU(q): x / max(|x|, 1e-12)
+      const float ik = raw_qk ? 1.f / fmaxf(sqrtf(nk), 1e-12f) : 1.f;
+      const float iq = raw_qk ? 1.f / fmaxf(sqrtf(nq), 1e-12f) : 1.f;
+      float bb = __ldg(beta + tok);
+      if (flags & kRawBeta) bb = sigmoid_f(bb);
+      s_ik[t] = ik;
+      s_iq[t] = iq;
+      s_kq[t] = kq * ik * iq;
+      s_beta[t] = bb;
     }
-    __syncthreads();
+  }
+  __syncthreads();
 
-    // Decay rows and accumulate partial r = S'^T k and p = S'^T q.
+  for (int t = 0; t < T; ++t) {
+    const int buf = t & 1;
     float4 r = make_float4(0.f, 0.f, 0.f, 0.f), p = r;
 #pragma unroll
     for (int i = 0; i < NI; ++i) {
       const int row = (warp + i * kWarps) * RPI + sub;
-      const float a = s_a[buf][row], kk = s_k[buf][row], qq = s_q[buf][row];
+      const float a = s_a[t][row], kk = s_k[t][row], qq = s_q[t][row];
       s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
       r.x = fmaf(s[i].x, kk, r.x); r.y = fmaf(s[i].y, kk, r.y);
       r.z = fmaf(s[i].z, kk, r.z); r.w = fmaf(s[i].w, kk, r.w);
@@ -121,7 +243,7 @@ decode_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* _
       p.z = fmaf(s[i].z, qq, p.z); p.w = fmaf(s[i].w, qq, p.w);
     }
 #pragma unroll
-    for (int off = LPR; off < 32; off <<= 1) {   // lanes holding the same columns
+    for (int off = LPR; off < 32; off <<= 1) {
       r.x += __shfl_xor_sync(0xffffffffu, r.x, off); r.y += __shfl_xor_sync(0xffffffffu, r.y, off);
       r.z += __shfl_xor_sync(0xffffffffu, r.z, off); r.w += __shfl_xor_sync(0xffffffffu, r.w, off);
       p.x += __shfl_xor_sync(0xffffffffu, p.x, off); p.y += __shfl_xor_sync(0xffffffffu, p.y, off);
@@ -132,19 +254,6 @@ decode_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* _
       s_red[buf][warp][1][cg] = p;
     }
     __syncthreads();
-
-    float kq = 0.f, nk2 = 0.f, nq2 = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      kq += s_sum[buf][w][0];
-      nk2 += s_sum[buf][w][1];
-      nq2 += s_sum[buf][w][2];
-    }
-    // L2 normalisation of SiLU(k), SiLU(q) folded into the reductions:
-    // x / max(|x|, 1e-12).
-    const float ik = raw_qk ? 1.f / fmaxf(sqrtf(nk2), 1e-12f) : 1.f;
-    const float iq = raw_qk ? 1.f / fmaxf(sqrtf(nq2), 1e-12f) : 1.f;
-    kq *= ik * iq;
     r = make_float4(0.f, 0.f, 0.f, 0.f);
     p = r;
 #pragma unroll
@@ -153,27 +262,25 @@ decode_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* _
       r.x += x.x; r.y += x.y; r.z += x.z; r.w += x.w;
       p.x += y.x; p.y += y.y; p.z += y.z; p.w += y.w;
     }
-    float bb = __ldg(beta + tok);
-    if (flags & kRawBeta) bb = sigmoid_f(bb);
-    const float rr[4] = {r.x * ik, r.y * ik, r.z * ik, r.w * ik};
-    const float pp[4] = {p.x * iq, p.y * iq, p.z * iq, p.w * iq};
-    float d[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      d[j] = bb * (Io<TIn>::load(v + tok * DV + col + j) - rr[j]);
-      if (warp == 0 && sub == 0) Io<TIn>::store(o + tok * DV + col + j, fmaf(kq, d[j], pp[j]));
+    const float ik = s_ik[t], iq = s_iq[t], kq = s_kq[t], bb = s_beta[t];
+    const float4 vv = *reinterpret_cast<const float4*>(&s_v[t][4 * cg]);
+    const float d[4] = {bb * (vv.x - r.x * ik), bb * (vv.y - r.y * ik), bb * (vv.z - r.z * ik),
+                        bb * (vv.w - r.w * ik)};
+    if (warp == 0 && sub == 0) {
+      const size_t tok = ((size_t)b * T + t) * H + h;
+      Io<TIn>::store(o + tok * DV + col, fmaf(kq, d[0], p.x * iq));
+      Io<TIn>::store(o + tok * DV + col + 1, fmaf(kq, d[1], p.y * iq));
+      Io<TIn>::store(o + tok * DV + col + 2, fmaf(kq, d[2], p.z * iq));
+      Io<TIn>::store(o + tok * DV + col + 3, fmaf(kq, d[3], p.w * iq));
     }
-    // S = S' + k d^T (k normalised).
 #pragma unroll
     for (int i = 0; i < NI; ++i) {
       const int row = (warp + i * kWarps) * RPI + sub;
-      const float kk = s_k[buf][row] * ik;
+      const float kk = s_k[t][row] * ik;
       s[i].x = fmaf(kk, d[0], s[i].x); s[i].y = fmaf(kk, d[1], s[i].y);
       s[i].z = fmaf(kk, d[2], s[i].z); s[i].w = fmaf(kk, d[3], s[i].w);
     }
   }
-
-  // Written once.
 #pragma unroll
   for (int i = 0; i < NI; ++i) {
     const int row = (warp + i * kWarps) * RPI + sub;
@@ -187,8 +294,12 @@ static cudaError_t launch_decode_t(const void* q, const void* k, const void* v,
                                    int n_heads, int T, int H, int gate, unsigned flags,
                                    cudaStream_t stream) {
   constexpr int kSplit = DV == 128 ? 2 : 1;
-  decode_kernel<TIn, DK, DV, kSplit><<<n_heads * kSplit, 256, 0, stream>>>(
-      (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, state, (TIn*)o, T, H, gate, flags);
+  if (T == 1 && gate == kGateChannel && flags == 0u)
+    decode_step_kernel<TIn, DK, DV, kSplit><<<n_heads * kSplit, 256, 0, stream>>>(
+        (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, state, (TIn*)o);
+  else
+    decode_multi_kernel<TIn, DK, DV, kSplit><<<n_heads * kSplit, 256, 0, stream>>>(
+        (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, state, (TIn*)o, T, H, gate, flags);
   return cudaGetLastError();
 }
 
