@@ -476,7 +476,7 @@ def bench_ours(args):
     var = None
     if not args.no_varlen:
         from gated_delta_rule_61_b200.inputs import varlen_lengths
-        lengths = varlen_lengths(64, 128, 32768, seed=0)
+        lengths = varlen_lengths(args.varlen_seqs, 128, args.varlen_max, seed=0)
         vin = prefill_inputs(1, 0, VARLEN["H"], 128, 128, dtype=torch.bfloat16, seed=2000 + rank,
                              init_std=0.1, lengths=lengths, device=dev)
         vo = torch.empty_like(vin["v"])
@@ -503,8 +503,9 @@ def bench_ours(args):
         vbytes = t_tot * VARLEN["H"] * BYTES_PER_HEAD_TOKEN + 2 * len(lengths) * VARLEN["H"] * 128 * 128 * 4
         vgbs = vbytes / (vms * 1e-3) / 1e9
         var = {"value": world * t_tot / (vms * 1e-3), "unit": "tokens/s", "ms_per_step": vms,
-               "workload": "KDA packed varlen prefill: 64 sequences log-uniform in [128, 32768] "
-                           "(%d tokens, longest %d), H=32, d=128, bf16, C=64" % (t_tot, max(lengths)),
+               "workload": "KDA packed varlen prefill: %d sequences log-uniform in [128, %d] "
+                           "(%d tokens, longest %d), H=32, d=128, bf16, C=64"
+                           % (len(lengths), args.varlen_max, t_tot, max(lengths)),
                "roofline": {"bound": "hbm", "achieved": vgbs, "peak": hbm, "unit": "GB/s",
                             "frac": vgbs / hbm, "traffic": kernel_traffic(VARLEN_PROFILE),
                             "peak_kind": peak_kind},
@@ -662,6 +663,10 @@ def main():
     ap.add_argument("--no-long", action="store_true")
     ap.add_argument("--no-forms", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--varlen-seqs", type=int, default=64,
+                    help="packed sequences of the varlen workload (a smaller case for profiling)")
+    ap.add_argument("--varlen-max", type=int, default=32768,
+                    help="longest sequence of the varlen workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--ref-budget", type=float, default=8.0)

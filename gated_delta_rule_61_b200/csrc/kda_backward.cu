@@ -30,8 +30,10 @@
 // slice of S at the start of every block of kBlk tokens to the workspace;
 // then, block by block from the last, the block's states are recomputed from
 // its checkpoint into a per-CTA scratch (kBlk x dk x 32 fp32, L2-resident)
-// and walked backwards. S' is recovered as S_t - k d^T with d kept from the
-// recomputation.
+// and walked backwards (the next token's state is loaded while the current
+// one is processed). S' is recovered as S_t - k d^T with d kept from the
+// recomputation. Each block's inputs are staged in shared memory once, so
+// the per-token steps wait on no global load.
 #include "kda_common.cuh"
 
 namespace kda {
@@ -61,7 +63,7 @@ __device__ __forceinline__ void red_add(float* p, float x) {
 }
 
 template <typename TIn, int DK, int DV>
-__global__ void __launch_bounds__(DK)
+__global__ void __launch_bounds__(DK, 2)
 backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
                 const float* __restrict__ log_alpha, const float* __restrict__ beta,
                 const float* __restrict__ init_state, const int32_t* __restrict__ cu_seqlens,
@@ -89,8 +91,32 @@ backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
   };
   float* scr = scratch + (size_t)blockIdx.x * kBlk * DK * kCols + (size_t)i * kCols;
 
+  // One block's inputs, staged once per block: key-row vectors (k, q, decay)
+  // and this slice's columns of v and d_o, beta per token.
+  __shared__ float s_k[kBlk][DK], s_q[kBlk][DK], s_a[kBlk][DK];
+  __shared__ float s_v[kBlk][kCols], s_do[kBlk][kCols];
+  __shared__ float s_beta[kBlk];
   __shared__ float s_part[kWarps][kCols];
   __shared__ float s_d[kBlk][kCols], s_vr[kBlk][kCols];   // d_j and v_j - r_j per token
+
+  auto stage = [&](long long tb, int nb, bool with_q) {
+    __syncthreads();   // the previous block's values are no longer read
+    for (int s = 0; s < nb; ++s) {
+      const size_t tok = (size_t)(tb + s) * H + head;
+      s_k[s][i] = Io<TIn>::load(k + tok * DK + i);
+      if (with_q) s_q[s][i] = Io<TIn>::load(q + tok * DK + i);
+      s_a[s][i] = gate == 0 ? expf(__ldg(log_alpha + tok * DK + i))
+                : gate == 1 ? expf(__ldg(log_alpha + tok)) : 1.f;
+    }
+    for (int e = i; e < nb * kCols; e += DK) {
+      const int s = e / kCols, j = e - (e / kCols) * kCols;
+      const size_t tok = (size_t)(tb + s) * H + head;
+      s_v[s][j] = Io<TIn>::load(v + tok * DV + col0 + j);
+      if (with_q) s_do[s][j] = Io<TIn>::load(d_o + tok * DV + col0 + j);
+    }
+    if (i < nb) s_beta[i] = __ldg(beta + (size_t)(tb + i) * H + head);
+    __syncthreads();
+  };
 
   const size_t state_off = ((size_t)seq * H + head) * DK * DV + (size_t)i * DV + col0;
   float S[kCols];
@@ -101,17 +127,10 @@ backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
     S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
   }
 
-  // Per-token row inputs of this thread (key row i) and column inputs.
-  auto decay = [&](size_t tok) {
-    return gate == 0 ? expf(__ldg(log_alpha + tok * DK + i))
-         : gate == 1 ? expf(__ldg(log_alpha + tok)) : 1.f;
-  };
-  // One forward step on S (row i, this slice's columns); leaves d_j and
-  // v_j - r_j in s_d[slot], s_vr[slot].
-  auto forward_step = [&](long long t, int slot) {
-    const size_t tok = (size_t)t * H + head;
-    const float a = decay(tok);
-    const float ki = Io<TIn>::load(k + tok * DK + i);
+  // One forward step of token slot s on S (row i, this slice's columns);
+  // leaves d_j and v_j - r_j in s_d[s], s_vr[s].
+  auto forward_step = [&](int s) {
+    const float a = s_a[s][i], ki = s_k[s][i];
     float part[kCols];
 #pragma unroll
     for (int j = 0; j < kCols; ++j) {
@@ -121,18 +140,17 @@ backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
     const float rl = warp_transpose_sum32(part, lane);
     s_part[warp][lane] = rl;
     __syncthreads();
-    const float bt = __ldg(beta + tok);
     if (warp == 0) {
       float r = 0.f;
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) r += s_part[w][lane];
-      const float vr = Io<TIn>::load(v + tok * DV + col0 + lane) - r;
-      s_vr[slot][lane] = vr;
-      s_d[slot][lane] = bt * vr;
+      const float vr = s_v[s][lane] - r;
+      s_vr[s][lane] = vr;
+      s_d[s][lane] = s_beta[s] * vr;
     }
     __syncthreads();
 #pragma unroll
-    for (int j = 0; j < kCols; ++j) S[j] = fmaf(ki, s_d[slot][j], S[j]);
+    for (int j = 0; j < kCols; ++j) S[j] = fmaf(ki, s_d[s][j], S[j]);
   };
 
   // Pass 1: forward over the sequence, checkpointing S at every block start.
@@ -141,10 +159,10 @@ backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
 #pragma unroll
     for (int j = 0; j < kCols; j += 4)
       __stcg(reinterpret_cast<float4*>(cp + j), make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]));
+    if (b + 1 == n_blk) break;
     const long long tb = t_begin + (long long)b * kBlk;
-    const int nb = (int)((t_end - tb) < kBlk ? (t_end - tb) : kBlk);
-    if (b + 1 < n_blk)
-      for (int s = 0; s < nb; ++s) forward_step(tb + s, 0);
+    stage(tb, kBlk, false);
+    for (int s = 0; s < kBlk; ++s) forward_step(s);
   }
 
   // Pass 2: blocks from the last; G = dL/dS.
@@ -158,6 +176,7 @@ backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
   for (int b = n_blk - 1; b >= 0; --b) {
     const long long tb = t_begin + (long long)b * kBlk;
     const int nb = (int)((t_end - tb) < kBlk ? (t_end - tb) : kBlk);
+    stage(tb, nb, true);
     const float* cp = ckpt_row(b);
 #pragma unroll
     for (int j = 0; j < kCols; j += 4) {
@@ -166,60 +185,63 @@ backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
     }
     // recompute the block, keeping S_t per token in the scratch
     for (int s = 0; s < nb; ++s) {
-      forward_step(tb + s, s);
+      forward_step(s);
       float* dst = scr + (size_t)s * DK * kCols;
 #pragma unroll
       for (int j = 0; j < kCols; j += 4)
         __stcg(reinterpret_cast<float4*>(dst + j), make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]));
     }
-    // reverse sweep
-    for (int s = nb - 1; s >= 0; --s) {
-      const long long t = tb + s;
-      const size_t tok = (size_t)t * H + head;
-      const float* src = scr + (size_t)s * DK * kCols;
+    // reverse sweep; S_t of the next token (s - 1) is loaded while this one
+    // is processed
+    float Sn[kCols];
+    {
+      const float* src = scr + (size_t)(nb - 1) * DK * kCols;
 #pragma unroll
       for (int j = 0; j < kCols; j += 4) {
         const float4 x = __ldcg(reinterpret_cast<const float4*>(src + j));
-        S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;   // S_t
+        Sn[j] = x.x; Sn[j + 1] = x.y; Sn[j + 2] = x.z; Sn[j + 3] = x.w;
       }
-      const float ki = Io<TIn>::load(k + tok * DK + i);
-      const float qi = Io<TIn>::load(q + tok * DK + i);
-      const float a = decay(tok);
-      const float bt = __ldg(beta + tok);
-      float dov[kCols];
+    }
+    for (int s = nb - 1; s >= 0; --s) {
 #pragma unroll
-      for (int j = 0; j < kCols; ++j) dov[j] = Io<TIn>::load(d_o + tok * DV + col0 + j);
+      for (int j = 0; j < kCols; ++j) S[j] = Sn[j];   // S_t
+      if (s > 0) {
+        const float* src = scr + (size_t)(s - 1) * DK * kCols;
+#pragma unroll
+        for (int j = 0; j < kCols; j += 4) {
+          const float4 x = __ldcg(reinterpret_cast<const float4*>(src + j));
+          Sn[j] = x.x; Sn[j + 1] = x.y; Sn[j + 2] = x.z; Sn[j + 3] = x.w;
+        }
+      }
+      const size_t tok = (size_t)(tb + s) * H + head;
+      const float ki = s_k[s][i], qi = s_q[s][i], a = s_a[s][i], bt = s_beta[s];
       // o_t = S_t^T q: G += q do^T; dq_i = sum_j S_t,ij do_j
       float dqi = 0.f;
       float part[kCols];
 #pragma unroll
       for (int j = 0; j < kCols; ++j) {
-        dqi = fmaf(S[j], dov[j], dqi);
-        G[j] = fmaf(qi, dov[j], G[j]);
+        const float doj = s_do[s][j];
+        dqi = fmaf(S[j], doj, dqi);
+        G[j] = fmaf(qi, doj, G[j]);
         part[j] = G[j] * ki;
       }
       // dd_j = sum_i G_ij k_i
       const float ddl = warp_transpose_sum32(part, lane);
       s_part[warp][lane] = ddl;
       __syncthreads();
-      float dd[kCols];
-#pragma unroll
-      for (int j = 0; j < kCols; ++j) {
-        float x = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) x += s_part[w][j];
-        dd[j] = x;
-      }
       // S_t = S' + k d^T; d = beta (v - r); r = S'^T k
       float dki = 0.f, dlai = 0.f, dbt = 0.f;
 #pragma unroll
       for (int j = 0; j < kCols; ++j) {
+        float ddj = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) ddj += s_part[w][j];
         const float dj = s_d[s][j];
         const float sp = fmaf(-ki, dj, S[j]);          // S'_ij
-        const float dr = -bt * dd[j];
+        const float dr = -bt * ddj;
         dki = fmaf(G[j], dj, dki);                     // G d
         dki = fmaf(sp, dr, dki);                       // S' dr
-        dbt = fmaf(dd[j], s_vr[s][j], dbt);
+        dbt = fmaf(ddj, s_vr[s][j], dbt);
         G[j] = fmaf(ki, dr, G[j]);                     // G'
         dlai = fmaf(sp, G[j], dlai);
         G[j] *= a;

@@ -219,7 +219,8 @@ __device__ __forceinline__ void cta_sync_tc() {
 // (their entries above the diagonal come out as exact zeros), level 2 fills
 // the two 16 x 16 blocks below them, level 3 the 32 x 32 block. Entries above
 // the diagonal outside the diagonal blocks are never read.
-__device__ __forceinline__ void invert_diag_block(const float* N, float* X, int t) {
+__device__ __forceinline__ void invert_diag_block(const float* N, float* X, uint8_t* tm,
+                                                  const float* s_beta, int t) {
   const int base = (t >> 4) * 16, col = t & 15;
   float x[16];
 #pragma unroll
@@ -236,15 +237,52 @@ __device__ __forceinline__ void invert_diag_block(const float* N, float* X, int 
   }
 #pragma unroll
   for (int rr = 0; rr < 16; ++rr) X[(base + rr) * kLd + base + col] = x[rr];
+  // T = X diag(beta) in bf16 (entries above the diagonal are exact zeros)
+  const float bc = s_beta[base + col];
+#pragma unroll
+  for (int rr = 0; rr < 16; ++rr)
+    *reinterpret_cast<__nv_bfloat16*>(tm + tc::sw128<2>(base + rr, base + col, 64)) =
+        __float2bfloat16_rn(x[rr] * bc);
 }
 
-__device__ __forceinline__ void invert_unit_lower64(const float* N, float* X, float* Z, int t) {
+// bf16 pair (r, j), (r, j + 1) of T, scaled by beta_j, beta_(j+1), into the
+// swizzled K-major T tile [r][j] (j even).
+__device__ __forceinline__ void store_t2(uint8_t* tm, const float* s_beta, int r, int j,
+                                         float x0, float x1) {
+  *reinterpret_cast<uint32_t*>(tm + tc::sw128<2>(r, j, 64)) =
+      pack_bf16x2(x0 * s_beta[j], x1 * s_beta[j + 1]);
+}
+
+// X = (I + N)^-1 as below, writing T = X diag(beta) (bf16, K-major [r][j],
+// the W/U MMA's operand) as each block of X is found: diagonal blocks in
+// level 1, the level-2 blocks, the level-3 block (which is not kept in fp32),
+// and zeros above the block diagonal (warps 2..7 while levels 1 and 2 run).
+// Ends without a CTA barrier: the caller's barrier publishes T.
+__device__ __forceinline__ void invert_unit_lower64(const float* N, float* X, float* Z,
+                                                    uint8_t* tm, const float* s_beta, int t) {
   // Levels 1 and 2 in warps 0 and 1: warp p inverts the diagonal blocks 2p
   // and 2p + 1, then fills block (2p + 1, 2p) below them with two 16 x 16 x 16
   // tf32 m16n8k8 products (tf32 rounding there is below the bf16 rounding T
   // receives next), so nothing outside the warp is waited for until level 3.
+  if (t >= 64 && t < 256) {
+    // zeros of T above the block diagonal: rows 0-15 x cols 16-63, rows
+    // 16-31 x cols 32-63, rows 32-47 x cols 48-63, in 16-byte chunks
+    const int idx = t - 64;
+    int r, c;
+    if (idx < 96) {
+      r = idx / 6;
+      c = 16 + (idx % 6) * 8;
+    } else if (idx < 160) {
+      r = 16 + (idx - 96) / 4;
+      c = 32 + ((idx - 96) % 4) * 8;
+    } else {
+      r = 32 + (idx - 160) / 2;
+      c = 48 + ((idx - 160) % 2) * 8;
+    }
+    *reinterpret_cast<uint4*>(tm + tc::sw128<2>(r, c, 64)) = make_uint4(0u, 0u, 0u, 0u);
+  }
   if (t < 64) {
-    invert_diag_block(N, X, t);
+    invert_diag_block(N, X, tm, s_beta, t);
     __syncwarp();
     const int p = t >> 5, lane = t & 31, gid = lane >> 2, tig = lane & 3;
     const int a = 32 * p, b = a + 16;
@@ -287,6 +325,8 @@ __device__ __forceinline__ void invert_unit_lower64(const float* N, float* X, fl
       const int xc = a + 8 * nt + 2 * tig;
       *reinterpret_cast<float2*>(X + (b + gid) * kLd + xc) = make_float2(-d[0], -d[1]);
       *reinterpret_cast<float2*>(X + (b + gid + 8) * kLd + xc) = make_float2(-d[2], -d[3]);
+      store_t2(tm, s_beta, b + gid, xc, -d[0], -d[1]);
+      store_t2(tm, s_beta, b + gid + 8, xc, -d[2], -d[3]);
     }
   }
   __syncthreads();
@@ -335,10 +375,9 @@ __device__ __forceinline__ void invert_unit_lower64(const float* N, float* X, fl
       mma_16x8x8_tf32(d, a, b);
     }
     const int xr = 32 + 16 * mt + gid, xc = 8 * nt + 2 * tig;
-    *reinterpret_cast<float2*>(X + xr * kLd + xc) = make_float2(-d[0], -d[1]);
-    *reinterpret_cast<float2*>(X + (xr + 8) * kLd + xc) = make_float2(-d[2], -d[3]);
+    store_t2(tm, s_beta, xr, xc, -d[0], -d[1]);
+    store_t2(tm, s_beta, xr + 8, xc, -d[2], -d[3]);
   }
-  __syncthreads();
 }
 
 // O^T (lane m, column r) of one chunk -> bf16 [r][m] in shared memory ->
@@ -800,12 +839,13 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     // ---- P2: Gram MMA (M=128, N=160, K=128) --------------------------------
     if (tid == 0) {
       constexpr uint32_t idesc = tc::make_idesc(1, 0, 0, 128, 160);
+      // base descriptors once; the k-steps add constant byte offsets (>> 4)
+      const uint64_t da0 = tc::make_desc(sbase + OFF_AG, 16, 1024);
+      const uint64_t db0 = tc::make_desc(sbase + OFF_BG, 16, 1024);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t da =
-            tc::make_desc(sbase + OFF_AG + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-        const uint64_t db =
-            tc::make_desc(sbase + OFF_BG + (ks >> 2) * 20480 + (ks & 3) * 32, 16, 1024);
+        const uint64_t da = da0 + (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
+        const uint64_t db = db0 + (uint64_t)(((ks >> 2) * 20480 + (ks & 3) * 32) >> 4);
         tc::mma_bf16_ss(tmem + TM_G, da, db, idesc, ks > 0 ? 1u : 0u);
       }
       tc::mma_commit(mbar);
@@ -921,20 +961,8 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       if (n >= step && warp >= 8)
         store_output_8w(tmem, lane_off, (warp >> 2) & 1, m, smem + OFF_SB, o,
                         t0 - (long long)step * C, C, H, head);
-      invert_unit_lower64(N, X, reinterpret_cast<float*>(smem + OFF_ZBUF), tid);
-      const int r = tid >> 3, j0 = (tid & 7) * 8;
-      uint32_t w[4];
-#pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        const int j = j0 + e;
-        const float2 xv = *reinterpret_cast<const float2*>(X + r * kLd + j);
-        const float2 bv = *reinterpret_cast<const float2*>(s_beta + j);
-        const float x0 = j <= r ? xv.x * bv.x : 0.f;
-        const float x1 = j + 1 <= r ? xv.y * bv.y : 0.f;
-        w[e >> 1] = pack_bf16x2(x0, x1);
-      }
-      *reinterpret_cast<uint4*>(smem + OFF_TM + tc::sw128<2>(r, j0, 64)) =
-          make_uint4(w[0], w[1], w[2], w[3]);
+      invert_unit_lower64(N, X, reinterpret_cast<float*>(smem + OFF_ZBUF), smem + OFF_TM,
+                          s_beta, tid);
     }
     tc::fence_async_smem();
     cta_sync_tc();
@@ -943,11 +971,14 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     // meanwhile S0 -> bf16 tile and the decay of the fp32 state -------------
     if (tid == 0) {
       constexpr uint32_t idesc = tc::make_idesc(1, 1, 0, 128, 64);
+      const uint64_t dw0 = tc::make_desc(sbase + OFF_BK, 8192, 1024);
+      const uint64_t du0 = tc::make_desc(sbase + OFF_VV, 8192, 1024);
+      const uint64_t dt0 = tc::make_desc(sbase + OFF_TM, 16, 1024);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
-        const uint64_t dw = tc::make_desc(sbase + OFF_BK + ks * 2048, 8192, 1024);
-        const uint64_t du = tc::make_desc(sbase + OFF_VV + ks * 2048, 8192, 1024);
-        const uint64_t dt = tc::make_desc(sbase + OFF_TM + ks * 32, 16, 1024);
+        const uint64_t dw = dw0 + (uint64_t)((ks * 2048) >> 4);
+        const uint64_t du = du0 + (uint64_t)((ks * 2048) >> 4);
+        const uint64_t dt = dt0 + (uint64_t)((ks * 32) >> 4);
         tc::mma_bf16_ss(tmem + TM_W, dw, dt, idesc, ks > 0 ? 1u : 0u);
         tc::mma_bf16_ss(tmem + TM_D, du, dt, idesc, ks > 0 ? 1u : 0u);
       }
@@ -1058,13 +1089,14 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     if (tid == 0) {
       constexpr uint32_t id_d = tc::make_idesc(1, 0, 1, 128, 64);
       constexpr uint32_t id_o = tc::make_idesc(1, 0, 0, 128, 64);
+      const uint64_t da0 = tc::make_desc(sbase + OFF_SB, 16, 1024);
+      const uint64_t dn0 = tc::make_desc(sbase + OFF_NW, 16384, 1024);
+      const uint64_t dq0 = tc::make_desc(sbase + OFF_QT, 16, 1024);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t da =
-            tc::make_desc(sbase + OFF_SB + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-        const uint64_t dn = tc::make_desc(sbase + OFF_NW + ks * 2048, 16384, 1024);
-        const uint64_t dq =
-            tc::make_desc(sbase + OFF_QT + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+        const uint64_t da = da0 + (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
+        const uint64_t dn = dn0 + (uint64_t)((ks * 2048) >> 4);
+        const uint64_t dq = dq0 + (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) >> 4);
         tc::mma_bf16_ss(tmem + TM_D, da, dn, id_d, 1u);
         tc::mma_bf16_ss(tmem + TM_O, da, dq, id_o, ks > 0 ? 1u : 0u);
       }
@@ -1086,13 +1118,13 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     if (tid == 0) {
       constexpr uint32_t id_s = tc::make_idesc(2, 0, 0, 128, 128);
       constexpr uint32_t id_o = tc::make_idesc(2, 0, 0, 128, 64);
+      const uint64_t dk0 = tc::make_desc(sbase + OFF_KT, 16, 1024);
+      const uint64_t dm0 = tc::make_desc(sbase + OFF_MQK, 16, 1024);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
         const uint32_t a_t = tmem + TM_D + ks * 8;
-        const uint64_t dk_ =
-            tc::make_desc(sbase + OFF_KT + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-        const uint64_t dm =
-            tc::make_desc(sbase + OFF_MQK + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+        const uint64_t dk_ = dk0 + (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
+        const uint64_t dm = dm0 + (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) >> 4);
         tc::mma_tf32_ts(tmem + TM_S, a_t, dk_, id_s, 1u);
         tc::mma_tf32_ts(tmem + TM_O, a_t, dm, id_o, 1u);
       }

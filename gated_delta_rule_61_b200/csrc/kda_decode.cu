@@ -68,6 +68,12 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
 
   float* S = state + (size_t)head * DK * DV;
 
+  // Launched with programmatic dependent launch, this grid can be scheduled
+  // while the previous kernel on the stream finishes; nothing is read before
+  // that kernel's writes are visible (it may have produced q, k, v or the
+  // state), so the wait comes first.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
   // Issue the state loads first: they are the bytes that matter.
   float4 s[NI];
 #pragma unroll
@@ -75,16 +81,20 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
     const int row = (warp + i * kWarps) * RPI + sub;
     s[i] = __ldcs(reinterpret_cast<const float4*>(S + (size_t)row * DV + col));
   }
+  float kk0 = 0.f, qq0 = 0.f, la0 = 0.f;
+  if (threadIdx.x < DK) {
+    kk0 = Io<TIn>::load(k + (size_t)head * DK + threadIdx.x);
+    qq0 = Io<TIn>::load(q + (size_t)head * DK + threadIdx.x);
+    la0 = __ldg(log_alpha + (size_t)head * DK + threadIdx.x);
+  }
 
   // Small per-head vectors: k, q, alpha = exp(log_alpha); k . q per warp.
   float kq_part = 0.f;
-  for (int i = threadIdx.x; i < DK; i += blockDim.x) {
-    const float kk = Io<TIn>::load(k + (size_t)head * DK + i);
-    const float qq = Io<TIn>::load(q + (size_t)head * DK + i);
-    s_k[i] = kk;
-    s_q[i] = qq;
-    s_a[i] = expf(__ldg(log_alpha + (size_t)head * DK + i));
-    kq_part += kk * qq;
+  if (threadIdx.x < DK) {
+    s_k[threadIdx.x] = kk0;
+    s_q[threadIdx.x] = qq0;
+    s_a[threadIdx.x] = expf(la0);
+    kq_part = kk0 * qq0;
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) kq_part += __shfl_xor_sync(0xffffffffu, kq_part, off);
@@ -146,6 +156,9 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
     s[i].z = fmaf(kk, d[2], s[i].z); s[i].w = fmaf(kk, d[3], s[i].w);
     __stcs(reinterpret_cast<float4*>(S + (size_t)row * DV + col), s[i]);
   }
+  // the next kernel on the stream may be scheduled now (its reads still wait
+  // for this grid to finish)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // Every other decode call (1 to 16 tokens, any gate form, prologue flags):
@@ -294,10 +307,21 @@ static cudaError_t launch_decode_t(const void* q, const void* k, const void* v,
                                    int n_heads, int T, int H, int gate, unsigned flags,
                                    cudaStream_t stream) {
   constexpr int kSplit = DV == 128 ? 2 : 1;
-  if (T == 1 && gate == kGateChannel && flags == 0u)
-    decode_step_kernel<TIn, DK, DV, kSplit><<<n_heads * kSplit, 256, 0, stream>>>(
-        (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, state, (TIn*)o);
-  else
+  if (T == 1 && gate == kGateChannel && flags == 0u) {
+    // programmatic dependent launch: scheduled while the previous kernel on
+    // the stream finishes (the kernel waits for it before reading anything)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(n_heads * kSplit));
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_step_kernel<TIn, DK, DV, kSplit>, (const TIn*)q,
+                              (const TIn*)k, (const TIn*)v, la, beta, state, (TIn*)o);
+  } else
     decode_multi_kernel<TIn, DK, DV, kSplit><<<n_heads * kSplit, 256, 0, stream>>>(
         (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, state, (TIn*)o, T, H, gate, flags);
   return cudaGetLastError();
