@@ -514,7 +514,9 @@ def bench_ours(args):
     # ---------------- long context: one 1M-token prefill, then graph-replayed decode ----------------
     lng = None
     if not args.no_long:
-        L = LONG
+        L = dict(LONG)
+        if args.long_tokens:
+            L["T"] = args.long_tokens
         lin = prefill_inputs(1, L["T"], L["H"], 128, 128, dtype=torch.bfloat16, seed=4000 + rank,
                              device=dev)
         lo = torch.empty_like(lin["v"])
@@ -661,6 +663,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-varlen", action="store_true")
     ap.add_argument("--no-long", action="store_true")
+    ap.add_argument("--long-tokens", type=int, default=0,
+                    help="tokens of the long-context prefill (default: the full workload)")
     ap.add_argument("--no-forms", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--varlen-seqs", type=int, default=64,

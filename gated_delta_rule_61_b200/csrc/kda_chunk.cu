@@ -52,10 +52,11 @@
 // Per chunk n: (P1) operand tiles from the chunk's gates and inputs; (P2)
 // Gram MMA, during which the next own chunk's inputs are loaded into
 // registers; (P3) rows of M_kk and M_qk; (P4) block inverse for X in warps
-// 0-7 while warps 8-15 move the previous own chunk's output to HBM; (P5) W^T
-// and U^T MMAs (with one CTA per chain, the state is copied to bf16 and
-// decayed in place meanwhile); -W to shared memory; with a ring, the state
-// is received here; (P7) D and the first part of O, during which the next
+// 0-7 while warps 8-15 move the previous own chunk's output to HBM and enter
+// the chunk's state (S0 to a bf16 tile, the fp32 state decayed in place;
+// with a ring, from the previous CTA's hand-over once it has arrived); (P5)
+// W^T and U^T MMAs; -W to shared memory; with a ring whose state arrived
+// after P4, the state is received here; (P7) D and the first part of O, during which the next
 // own chunk's gates (cumulative sums, sub-chunk ends, decay) are formed
 // (with four CTAs per chain, where P7 is on the ring's critical path, at
 // the start of that chunk's P1 instead); (P8) tf32 state update and output
@@ -95,7 +96,8 @@ constexpr uint32_t MISC_GAMMA = 0, MISC_BETA = 512, MISC_PAIR = 1280,
                    MISC_GF = 17664, MISC_GL = 19712, MISC_MBAR = 21760, MISC_FULL = 21776,
                    MISC_TMEM = 21784, MISC_TOT4 = 21792,
                    MISC_NORM = 23840,   // raw q/k: per-warp partial squared norms [16][16]
-                   MISC_BARA = 24864;   // mbarrier of the k/v tensor-map copies
+                   MISC_BARA = 24864,   // mbarrier of the k/v tensor-map copies
+                   MISC_FLAG = 24872;   // P4: the ring's entering state was already handed over
 constexpr uint32_t kSmemBytes = OFF_MISC + 24880 + 1024;
 // The next own chunk's raw k and v land by tensor-map copies (128B-swizzled
 // [row][channel] tiles, the operand tiles' layout): k in the K e^g tile (P1
@@ -222,18 +224,18 @@ __device__ __forceinline__ void cta_sync_tc() {
 __device__ __forceinline__ void invert_diag_block(const float* N, float* X, uint8_t* tm,
                                                   const float* s_beta, int t) {
   const int base = (t >> 4) * 16, col = t & 15;
+  // Column col of the block's inverse by right-looking substitution: once
+  // x[j] is final, every later row subtracts its term N[r][j] x[j], so the
+  // dependent chain is one FMA per row while the other updates (and all the
+  // loads of N) proceed in parallel.
   float x[16];
 #pragma unroll
-  for (int rr = 0; rr < 16; ++rr) {
-    const float* nr = N + (base + rr) * kLd + base;
-    float a0 = rr == col ? 1.f : 0.f, a1 = 0.f;
+  for (int rr = 0; rr < 16; ++rr) x[rr] = rr == col ? 1.f : 0.f;
+  const float* nb = N + base * kLd + base;
 #pragma unroll
-    for (int jj = 0; jj + 1 < rr; jj += 2) {
-      a0 -= nr[jj] * x[jj];
-      a1 -= nr[jj + 1] * x[jj + 1];
-    }
-    if (rr & 1) a0 -= nr[rr - 1] * x[rr - 1];
-    x[rr] = a0 + a1;
+  for (int j = 0; j < 15; ++j) {
+#pragma unroll
+    for (int rr = j + 1; rr < 16; ++rr) x[rr] = fmaf(-nb[rr * kLd + j], x[j], x[rr]);
   }
 #pragma unroll
   for (int rr = 0; rr < 16; ++rr) X[(base + rr) * kLd + base + col] = x[rr];
@@ -423,6 +425,51 @@ __device__ __forceinline__ void store_output_8w(uint32_t tmem, uint32_t lane_off
   }
 }
 
+// 32 columns [cb, cb + 32) of row m of the entering state S0 (fp32, in s):
+// bf16 into the S0 tile (swizzled K-major [m][c]), decayed by gamma into
+// tensor memory at taddr.
+__device__ __forceinline__ void state_tile_and_decay(uint32_t taddr, int m, int cb, uint8_t* smem,
+                                                     const float* s_gamma, float* s) {
+#pragma unroll
+  for (int h8 = 0; h8 < 4; ++h8) {
+    uint32_t p[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) p[e] = pack_bf16x2(s[h8 * 8 + 2 * e], s[h8 * 8 + 2 * e + 1]);
+    *reinterpret_cast<uint4*>(smem + OFF_SB + tc::sw128<2>(m, cb + h8 * 8, 128)) =
+        make_uint4(p[0], p[1], p[2], p[3]);
+  }
+#pragma unroll
+  for (int i = 0; i < 32; ++i) s[i] *= s_gamma[cb + i];
+  tc::tmem_st16(taddr, s);
+  tc::tmem_st16(taddr + 16, s + 16);
+}
+
+// The entering state of a chunk, by warps 8-15 (two per lane quadrant, 64
+// columns [64 half, +64) each): from tensor memory, or (slot != nullptr)
+// from the chain's hand-over slot.
+__device__ __forceinline__ void enter_state(uint32_t tmem, uint32_t lane_off, int m, int half,
+                                            uint8_t* smem, const float* s_gamma,
+                                            const float* slot) {
+#pragma unroll 1
+  for (int hh = 0; hh < 2; ++hh) {
+    const int cb = half * 64 + hh * 32;
+    const uint32_t tb = tmem + lane_off + TM_S + cb;
+    float s[32];
+    if (slot) {
+      const float4* sl = reinterpret_cast<const float4*>(slot);
+#pragma unroll
+      for (int v4 = 0; v4 < 8; ++v4) {
+        const float4 x = __ldcg(sl + xfer_chunk(m, cb / 4 + v4));
+        s[4 * v4] = x.x; s[4 * v4 + 1] = x.y; s[4 * v4 + 2] = x.z; s[4 * v4 + 3] = x.w;
+      }
+    } else {
+      tc::tmem_ld32(tb, s);
+    }
+    state_tile_and_decay(tb, m, cb, smem, s_gamma, s);
+  }
+  tc::tmem_wait_st();
+}
+
 // kGate: 0 = one decay per key channel (log_alpha [.., H, dk]), 1 = one per
 // token (log_alpha [.., H], the same value on every channel), 2 = none.
 // kRawQK: q and k are raw projections; each token's vectors become
@@ -437,7 +484,8 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
                const int32_t* __restrict__ cu_seqlens, const int32_t* __restrict__ order,
                int T, int H, __nv_bfloat16* __restrict__ o, float* final_state, float* xfer,
                unsigned flags, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v) {
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q,
+               const __grid_constant__ CUtensorMap tm_la) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -856,20 +904,27 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     // tiles) and warm L2 with the inputs of the own chunk after it.
     if (n + step < n_chunks) load_rows(n + step);
     if (n + 2 * step < n_chunks) {
+      // q, k, v and the per-channel gates by tensor-map prefetches (one
+      // thread, a few box requests); beta and a per-token gate row by row.
       const long long t1 = t0 + (long long)(2 * step) * C;
-      const int row = tid >> 3, part = tid & 7;
-      if (t1 + row < t_end) {
-        const size_t tok = (size_t)(t1 + row) * H + head;
-        if (part < 2) tc::prefetch_l2(q + tok * DK + 64 * part);
-        else if (part < 4) tc::prefetch_l2(k + tok * DK + 64 * (part - 2));
-        else if (part < 6) tc::prefetch_l2(v + tok * DV + 64 * (part - 4));
-        else if (kGate == 0) tc::prefetch_l2(log_alpha + tok * DK + 64 * (part - 6));
-        if (kGate == 0 && part == 6) tc::prefetch_l2(log_alpha + tok * DK + 32);
-        if (kGate == 1 && part == 6) tc::prefetch_l2(log_alpha + tok);
-        if (part == 7) {
-          if (kGate == 0) tc::prefetch_l2(log_alpha + tok * DK + 96);
-          tc::prefetch_l2(beta + tok);
+      const int z1 = (int)t1;
+      if (tid == 32) {
+#pragma unroll
+        for (int x = 0; x < 128; x += 64) {
+          tc::prefetch_box_3d(&tm_q, x, head, z1);
+          tc::prefetch_box_3d(&tm_k, x, head, z1);
+          tc::prefetch_box_3d(&tm_v, x, head, z1);
         }
+        if constexpr (kGate == 0) {
+#pragma unroll
+          for (int x = 0; x < 128; x += 32) tc::prefetch_box_3d(&tm_la, x, head, z1);
+        }
+      }
+      const int row = tid - 64;
+      if (row >= 0 && row < C && t1 + row < t_end) {
+        const size_t tok = (size_t)(t1 + row) * H + head;
+        tc::prefetch_l2(beta + tok);
+        if (kGate == 1) tc::prefetch_l2(log_alpha + tok);
       }
     }
     ok = cta_wait(mbar, phase, 1);
@@ -951,24 +1006,44 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     cta_sync_tc();
 
     // ---- P4: X = (I + N)^-1; T = X diag(beta) -> bf16 -------------------
+    // Warps 0-7 run the solve. Meanwhile warps 8-15 move the previous own
+    // chunk's output to HBM (staged in the gate-scan scratch, idle until the
+    // next gate scan), then prepare this chunk's entering state: the S0 bf16
+    // tile for the D/O MMA and the decayed fp32 state in tensor memory, from
+    // tensor memory (one CTA per chain, or a ring's first chunk), or from the
+    // chain's hand-over slot when the previous CTA of the ring has already
+    // handed it over (otherwise every warp receives it after the W/U MMA).
+    bool received = false;
     {
       const float* N = reinterpret_cast<const float*>(smem + OFF_NMAT);
       float* X = reinterpret_cast<float*>(smem + OFF_XMAT);
-      // Meanwhile warps 8..15 move the previous chunk's output to HBM (staged
-      // in the S0 bf16 tile, which is dead until P5). (Also copying and
-      // decaying the state there, to shorten P5, was measured slower: it
-      // delays the solve's first barrier more than it saves.)
-      if (n >= step && warp >= 8)
-        store_output_8w(tmem, lane_off, (warp >> 2) & 1, m, smem + OFF_SB, o,
-                        t0 - (long long)step * C, C, H, head);
+      int* s_flag = reinterpret_cast<int*>(smem + OFF_MISC + MISC_FLAG);
+      if (warp >= 8) {
+        const int half = (warp >> 2) & 1;
+        if (n >= step)
+          store_output_8w(tmem, lane_off, half, m, smem + OFF_MISC + MISC_PAIR, o,
+                          t0 - (long long)step * C, C, H, head);
+        bool from_slot = false;
+        if (kPair && n > 0) {
+          if (tid == 256) *s_flag = tc::mbar_test_wait_cluster(mbar_full, full_phase) ? 1 : 0;
+          asm volatile("bar.sync 2, 256;" ::: "memory");
+          from_slot = *s_flag != 0;
+        }
+        if (!(kPair && n > 0) || from_slot)
+          enter_state(tmem, lane_off, m, half, smem, s_gamma,
+                      from_slot ? xfer + xfer_off : nullptr);
+      }
       invert_unit_lower64(N, X, reinterpret_cast<float*>(smem + OFF_ZBUF), smem + OFF_TM,
                           s_beta, tid);
+      tc::fence_async_smem();
+      cta_sync_tc();
+      if (kPair && n > 0) received = *s_flag != 0;
+      if (received) full_phase ^= 1;
     }
-    tc::fence_async_smem();
-    cta_sync_tc();
 
     // ---- P5: W^T = (K e^g)^T T^T and U^T = V^T T^T (M=128, N=64, K=64);
-    // meanwhile S0 -> bf16 tile and the decay of the fp32 state -------------
+    // then -W^T to shared memory and, in a ring whose state was not yet
+    // handed over in P4, the entering state from the hand-over slot --------
     if (tid == 0) {
       constexpr uint32_t idesc = tc::make_idesc(1, 1, 0, 128, 64);
       const uint64_t dw0 = tc::make_desc(sbase + OFF_BK, 8192, 1024);
@@ -985,50 +1060,7 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       tc::mma_commit(mbar);
       pend_mma = true;
     }
-    const bool receive = kPair && n > 0;
-    if (!receive) {
-      // S -> bf16 tile and in-place decay (16 columns at a time in the
-      // one-CTA variant, where that keeps its registers within budget).
-      if constexpr (kRing == 1) {
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const uint32_t tb = tmem + lane_off + TM_S + grp * 32 + hh * 16;
-          float s[16];
-          tc::tmem_ld16(tb, s);
-          const int cb = grp * 32 + hh * 16;
-#pragma unroll
-          for (int h8 = 0; h8 < 2; ++h8) {
-            uint32_t p[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) p[e] = pack_bf16x2(s[h8 * 8 + 2 * e], s[h8 * 8 + 2 * e + 1]);
-            *reinterpret_cast<uint4*>(smem + OFF_SB + tc::sw128<2>(m, cb + h8 * 8, 128)) =
-                make_uint4(p[0], p[1], p[2], p[3]);
-          }
-#pragma unroll
-          for (int i = 0; i < 16; ++i) s[i] *= s_gamma[cb + i];
-          tc::tmem_st16(tb, s);
-        }
-        tc::tmem_wait_st();
-      } else {
-        const uint32_t tb = tmem + lane_off + TM_S + grp * 32;
-        float s[32];
-        tc::tmem_ld32(tb, s);
-        const int cb = grp * 32;
-#pragma unroll
-        for (int h8 = 0; h8 < 4; ++h8) {
-          uint32_t p[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) p[e] = pack_bf16x2(s[h8 * 8 + 2 * e], s[h8 * 8 + 2 * e + 1]);
-          *reinterpret_cast<uint4*>(smem + OFF_SB + tc::sw128<2>(m, cb + h8 * 8, 128)) =
-              make_uint4(p[0], p[1], p[2], p[3]);
-        }
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[i] *= s_gamma[cb + i];
-        tc::tmem_st16(tb, s);
-        tc::tmem_st16(tb + 16, s + 16);
-        tc::tmem_wait_st();
-      }
-    }
+    const bool receive = kPair && n > 0 && !received;
     ok = cta_wait(mbar, phase, 2);
     if (!ok) break;
     pend_mma = false;
@@ -1067,19 +1099,7 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         const float4 x = __ldcg(slot + xfer_chunk(m, cb / 4 + v4));
         s[4 * v4] = x.x; s[4 * v4 + 1] = x.y; s[4 * v4 + 2] = x.z; s[4 * v4 + 3] = x.w;
       }
-#pragma unroll
-      for (int h8 = 0; h8 < 4; ++h8) {
-        uint32_t p[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) p[e] = pack_bf16x2(s[h8 * 8 + 2 * e], s[h8 * 8 + 2 * e + 1]);
-        *reinterpret_cast<uint4*>(smem + OFF_SB + tc::sw128<2>(m, cb + h8 * 8, 128)) =
-            make_uint4(p[0], p[1], p[2], p[3]);
-      }
-#pragma unroll
-      for (int i = 0; i < 32; ++i) s[i] *= s_gamma[cb + i];
-      const uint32_t tb = tmem + lane_off + TM_S + grp * 32;
-      tc::tmem_st16(tb, s);
-      tc::tmem_st16(tb + 16, s + 16);
+      state_tile_and_decay(tmem + lane_off + TM_S + grp * 32, m, grp * 32, smem, s_gamma, s);
       tc::tmem_wait_st();
     }
     tc::fence_async_smem();
@@ -1170,7 +1190,8 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     const int n_mine = rank + step * ((n_chunks - 1 - rank) / step);   // this CTA's last chunk
     const long long t_last = t_begin + (long long)n_mine * C;
     const int L_last = (int)((t_end - t_last) < C ? (t_end - t_last) : C);
-    store_output(tmem, lane_off, grp, m, smem + OFF_SB, o, t_last, L_last, H, head);
+    store_output(tmem, lane_off, grp, m, smem + OFF_MISC + MISC_PAIR, o, t_last, L_last, H,
+                 head);
   }
   const bool owns_final = n_chunks > 0 ? ((n_chunks - 1) % step == rank) : rank == 0;
   if (ok && final_state && owns_final) {
@@ -1271,7 +1292,7 @@ struct ChunkArgs {
   __nv_bfloat16* o;
   float *sT, *xfer;
   unsigned flags;
-  CUtensorMap tm_k, tm_v;
+  CUtensorMap tm_k, tm_v, tm_q, tm_la;   // tm_q, tm_la: L2 prefetch only
 };
 
 // cuTensorMapEncodeTiled, reached through the runtime's driver entry point
@@ -1329,14 +1350,14 @@ static cudaError_t launch_variant(const ChunkArgs& a, long long chains, int ring
     if (ring == 4)
       return cudaLaunchKernelEx(&cfg, chunk64_kernel<4, kGate, kRaw>, a.q, a.k, a.v, a.la,
                                 a.beta, a.s0, a.cu, a.order, a.T, a.H, a.o, a.sT, a.xfer,
-                                a.flags, a.tm_k, a.tm_v);
+                                a.flags, a.tm_k, a.tm_v, a.tm_q, a.tm_la);
     return cudaLaunchKernelEx(&cfg, chunk64_kernel<2, kGate, kRaw>, a.q, a.k, a.v, a.la,
                               a.beta, a.s0, a.cu, a.order, a.T, a.H, a.o, a.sT, a.xfer,
-                              a.flags, a.tm_k, a.tm_v);
+                              a.flags, a.tm_k, a.tm_v, a.tm_q, a.tm_la);
   }
   chunk64_kernel<1, kGate, kRaw><<<(unsigned)chains, kThreads, kSmemBytes, stream>>>(
       a.q, a.k, a.v, a.la, a.beta, a.s0, a.cu, a.order, a.T, a.H, a.o, a.sT, nullptr, a.flags,
-      a.tm_k, a.tm_v);
+      a.tm_k, a.tm_v, a.tm_q, a.tm_la);
   return cudaGetLastError();
 }
 
@@ -1389,11 +1410,17 @@ cudaError_t launch_chunk64(const void* q, const void* k, const void* v, const fl
   const long long tokens = cu ? (long long)T : (long long)n_seq * T;
   if (tokens == 0) {
     memset(&a.tm_k, 0, sizeof(CUtensorMap));   // no chunk to load: never read
-    a.tm_v = a.tm_k;
+    a.tm_v = a.tm_q = a.tm_la = a.tm_k;
     return launch_variant<2, false>(a, chains, 1, stream);   // initial -> final states
   }
   if ((e1 = encode_rows(enc, &a.tm_k, k, true, tokens, H)) != cudaSuccess) return e1;
   if ((e1 = encode_rows(enc, &a.tm_v, v, true, tokens, H)) != cudaSuccess) return e1;
+  if ((e1 = encode_rows(enc, &a.tm_q, q, true, tokens, H)) != cudaSuccess) return e1;
+  if (gate == 0) {
+    if ((e1 = encode_rows(enc, &a.tm_la, la, false, tokens, H)) != cudaSuccess) return e1;
+  } else {
+    a.tm_la = a.tm_q;   // no per-channel gate tensor: never read
+  }
   // Few chains: R = 4 or 2 CTAs per chain (chunks round-robin), all in one
   // wave; the state passes between them through the chain's xfer slot.
   const int ring = (xfer && 2 * chains <= n_sm) ? (4 * chains <= n_sm ? 4 : 2) : 1;

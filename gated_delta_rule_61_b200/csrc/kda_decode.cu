@@ -42,10 +42,13 @@ __device__ __forceinline__ float decay_from(float g, unsigned flags) {
 // CTA (head, slice) owns value columns [slice * DV / SPLIT, +DV / SPLIT).
 // Within a CTA each lane owns one 4-column group; LPR = columns / 4 lanes
 // cover a row, so a warp instruction reads RPI = 32 / LPR whole rows (512
-// contiguous bytes per warp for 128 columns). 64 registers per thread keep
-// 2 * SPLIT CTAs per SM in flight.
+// contiguous bytes per warp for 128 columns). With SPLIT >= 2, 64 registers
+// per thread keep four CTAs per SM in flight.
+template <int SPLIT>
+constexpr int decode_min_blocks() { return SPLIT == 1 ? 2 : 4; }
+
 template <typename TIn, int DK, int DV, int SPLIT>
-__global__ void __launch_bounds__(256, 2 * SPLIT)
+__global__ void __launch_bounds__(256, decode_min_blocks<SPLIT>())
 decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                    const TIn* __restrict__ v, const float* __restrict__ log_alpha,
                    const float* __restrict__ beta, float* __restrict__ state,
@@ -168,7 +171,7 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
 // overlaps those loads with the state loads. The token loop then needs one
 // CTA barrier per token (the cross-warp part of r and p, double-buffered).
 template <typename TIn, int DK, int DV, int SPLIT>
-__global__ void __launch_bounds__(256, 2 * SPLIT)
+__global__ void __launch_bounds__(256, decode_min_blocks<SPLIT>())
 decode_multi_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                     const TIn* __restrict__ v, const float* __restrict__ log_alpha,
                     const float* __restrict__ beta, float* __restrict__ state,
@@ -203,8 +206,13 @@ decode_multi_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
   // Stage the tokens: warp w takes tokens w, w + 8.
   for (int t = warp; t < T; t += kWarps) {
     const size_t tok = ((size_t)b * T + t) * H + h;
-    float kq = 0.f, nk = 0.f, nq = 0.f;
-    for (int i = lane; i < DK; i += 32) {
+    // k . q is summed in the plain step's order (a warp tree over each 32
+    // channels, then the groups in turn), so a call over T tokens matches T
+    // single-token calls bit for bit.
+    float kqg[DK / 32], nk = 0.f, nq = 0.f;
+#pragma unroll
+    for (int g = 0; g < DK / 32; ++g) {
+      const int i = lane + 32 * g;
       float kk = Io<TIn>::load(k + tok * DK + i);
       float qq = Io<TIn>::load(q + tok * DK + i);
       if (raw_qk) {
@@ -219,15 +227,19 @@ decode_multi_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
       if (gate == kGateChannel) a = decay_from(__ldg(log_alpha + tok * DK + i), flags);
       else if (gate == kGateScalar) a = decay_from(__ldg(log_alpha + tok), flags);
       s_a[t][i] = a;
-      kq = fmaf(kk, qq, kq);
+      kqg[g] = kk * qq;
     }
     for (int j = lane; j < CW; j += 32) s_v[t][j] = Io<TIn>::load(v + tok * DV + slice * CW + j);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
-      kq += __shfl_xor_sync(0xffffffffu, kq, off);
+#pragma unroll
+      for (int g = 0; g < DK / 32; ++g) kqg[g] += __shfl_xor_sync(0xffffffffu, kqg[g], off);
       nk += __shfl_xor_sync(0xffffffffu, nk, off);
       nq += __shfl_xor_sync(0xffffffffu, nq, off);
     }
+    float kq = 0.f;
+#pragma unroll
+    for (int g = 0; g < DK / 32; ++g) kq += kqg[g];
     if (lane == 0) {
       // L2 normalisation of SiLU(k), SiLU(q): x / max(|x|, 1e-12)
       const float ik = raw_qk ? 1.f / fmaxf(sqrtf(nk), 1e-12f) : 1.f;
@@ -301,12 +313,11 @@ decode_multi_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
   }
 }
 
-template <typename TIn, int DK, int DV>
-static cudaError_t launch_decode_t(const void* q, const void* k, const void* v,
-                                   const float* la, const float* beta, float* state, void* o,
-                                   int n_heads, int T, int H, int gate, unsigned flags,
-                                   cudaStream_t stream) {
-  constexpr int kSplit = DV == 128 ? 2 : 1;
+template <typename TIn, int DK, int DV, int kSplit>
+static cudaError_t launch_decode_split(const void* q, const void* k, const void* v,
+                                       const float* la, const float* beta, float* state,
+                                       void* o, int n_heads, int T, int H, int gate,
+                                       unsigned flags, cudaStream_t stream) {
   if (T == 1 && gate == kGateChannel && flags == 0u) {
     // programmatic dependent launch: scheduled while the previous kernel on
     // the stream finishes (the kernel waits for it before reading anything)
@@ -321,10 +332,27 @@ static cudaError_t launch_decode_t(const void* q, const void* k, const void* v,
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, decode_step_kernel<TIn, DK, DV, kSplit>, (const TIn*)q,
                               (const TIn*)k, (const TIn*)v, la, beta, state, (TIn*)o);
-  } else
-    decode_multi_kernel<TIn, DK, DV, kSplit><<<n_heads * kSplit, 256, 0, stream>>>(
-        (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, state, (TIn*)o, T, H, gate, flags);
+  }
+  decode_multi_kernel<TIn, DK, DV, kSplit><<<n_heads * kSplit, 256, 0, stream>>>(
+      (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, state, (TIn*)o, T, H, gate, flags);
   return cudaGetLastError();
+}
+
+// Value slices per head: 2 (dv = 128) or 1 (dv = 64) fill the GPU once there
+// are a few hundred CTAs; with fewer heads (small-batch decode, latency-bound)
+// 16-column slices spread the state over eight or four times as many SMs.
+constexpr int kFewHeads = 128;
+
+template <typename TIn, int DK, int DV>
+static cudaError_t launch_decode_t(const void* q, const void* k, const void* v,
+                                   const float* la, const float* beta, float* state, void* o,
+                                   int n_heads, int T, int H, int gate, unsigned flags,
+                                   cudaStream_t stream) {
+  if (n_heads < kFewHeads)
+    return launch_decode_split<TIn, DK, DV, DV / 16>(q, k, v, la, beta, state, o, n_heads, T,
+                                                     H, gate, flags, stream);
+  return launch_decode_split<TIn, DK, DV, DV == 128 ? 2 : 1>(q, k, v, la, beta, state, o,
+                                                             n_heads, T, H, gate, flags, stream);
 }
 
 template <typename TIn>
