@@ -16,20 +16,22 @@
 //     dlog_alpha_i = sum_j S'_ij G'_ij;         G = Diag(a) G'
 // and dL/dS_0 = G at the end.
 //
-// Layout: one CTA per (sequence, head, 32-column slice of dv); thread i owns
-// key row i of the slice's 32 columns of S and of G (registers). Sums over
+// Layout: one CTA per (sequence, head, slice of kCols value columns: 32, or
+// 8 when chains are few, so that enough CTAs are resident to hide the
+// per-token latency); thread i owns key row i of the slice's columns of S
+// and of G (registers). Sums over
 // the value columns (dq, dk, dlog_alpha) stay inside a thread; the two sums
 // over key rows per token (r in the recomputation, dd in the reverse step)
 // are a halving-exchange reduction over the warp's lanes plus one shared-
 // memory exchange across warps. Column slices of one head add their partial
-// dq, dk, dlog_alpha and dbeta into the fp32 outputs (red.add; the four
-// slices' order is not fixed, so these gradients can differ between runs in
-// the last bits). dv and dL/dS_0 are written by their slice alone.
+// dq, dk, dlog_alpha and dbeta into the fp32 outputs (red.add; the slices'
+// order is not fixed, so these gradients can differ between runs in the
+// last bits). dv and dL/dS_0 are written by their slice alone.
 //
 // The states are not stored per token: a first forward pass writes the
 // slice of S at the start of every block of kBlk tokens to the workspace;
 // then, block by block from the last, the block's states are recomputed from
-// its checkpoint into a per-CTA scratch (kBlk x dk x 32 fp32, L2-resident)
+// its checkpoint into a per-CTA scratch (kBlk x dk x kCols fp32, L2-resident)
 // and walked backwards (the next token's state is loaded while the current
 // one is processed). S' is recovered as S_t - k d^T with d kept from the
 // recomputation. Each block's inputs are staged in shared memory once, so
@@ -40,13 +42,17 @@ namespace kda {
 namespace bwd {
 
 constexpr int kBlk = 16;       // tokens per checkpoint block
-constexpr int kCols = 32;      // value columns per CTA
+constexpr int kColsWide = 32, kColsNarrow = 8;   // value columns per CTA
 
-// Halving-exchange sum of 32 per-lane vectors of 32 values over the warp:
-// on return v[0] of lane l holds the warp sum of value l.
-__device__ __forceinline__ float warp_transpose_sum32(float* v, int lane) {
+// Sum over the warp of 32 per-lane vectors of N values (N a power of two,
+// at most 32): halving exchanges over offsets N/2 .. 1 (a lane keeps the
+// half of its values selected by its lane bit and adds the partner's copy of
+// that half), then plain exchanges over offsets N .. 16; lane l returns the
+// warp sum of value l % N.
+template <int N>
+__device__ __forceinline__ float warp_transpose_sum(float* v, int lane) {
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) {
+  for (int off = N / 2; off >= 1; off >>= 1) {
     const bool up = lane & off;
 #pragma unroll
     for (int j = 0; j < off; ++j) {
@@ -55,15 +61,18 @@ __device__ __forceinline__ float warp_transpose_sum32(float* v, int lane) {
       v[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
     }
   }
-  return v[0];
+  float x = v[0];
+#pragma unroll
+  for (int off = N; off < 32; off <<= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
 }
 
 __device__ __forceinline__ void red_add(float* p, float x) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(x) : "memory");
 }
 
-template <typename TIn, int DK, int DV>
-__global__ void __launch_bounds__(DK, 2)
+template <typename TIn, int DK, int DV, int kCols>
+__global__ void __launch_bounds__(DK, kCols == kColsNarrow ? 1024 / DK : 2)
 backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
                 const float* __restrict__ log_alpha, const float* __restrict__ beta,
                 const float* __restrict__ init_state, const int32_t* __restrict__ cu_seqlens,
@@ -137,10 +146,10 @@ backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
       S[j] *= a;
       part[j] = S[j] * ki;
     }
-    const float rl = warp_transpose_sum32(part, lane);
-    s_part[warp][lane] = rl;
+    const float rl = warp_transpose_sum<kCols>(part, lane);
+    if (lane < kCols) s_part[warp][lane] = rl;
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 0 && lane < kCols) {
       float r = 0.f;
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) r += s_part[w][lane];
@@ -226,8 +235,8 @@ backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
         part[j] = G[j] * ki;
       }
       // dd_j = sum_i G_ij k_i
-      const float ddl = warp_transpose_sum32(part, lane);
-      s_part[warp][lane] = ddl;
+      const float ddl = warp_transpose_sum<kCols>(part, lane);
+      if (lane < kCols) s_part[warp][lane] = ddl;
       __syncthreads();
       // S_t = S' + k d^T; d = beta (v - r); r = S'^T k
       float dki = 0.f, dlai = 0.f, dbt = 0.f;
@@ -250,7 +259,7 @@ backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
       red_add(dk + tok * DK + i, dki);
       if (gate == 0) red_add(dla + tok * DK + i, dlai);
       if (i == 0) red_add(dbeta + tok, dbt);
-      if (warp == 0) {
+      if (warp == 0 && lane < kCols) {
         float x = 0.f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) x += s_part[w][lane];
@@ -276,13 +285,13 @@ backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
 }  // namespace bwd
 
 // Workspace: checkpoints (floor(tokens / 16) + n_seq + 1 blocks per head, each
-// dk x dv fp32) and one 16 x dk x 32 fp32 scratch per CTA, 256-byte aligned.
+// dk x dv fp32) and one 16 x dk x kCols fp32 scratch per CTA (16 x dk x dv
+// per head whatever the slice width), 256-byte aligned.
 size_t backward_workspace_bytes(int n_seq, long long tokens, int H, int dk, int dv) {
   if (n_seq <= 0 || H <= 0) return 0;
   const size_t blocks = (size_t)(tokens / bwd::kBlk) + (size_t)n_seq + 1;
   const size_t ck = blocks * (size_t)H * dk * dv * sizeof(float);
-  const size_t ctas = (size_t)n_seq * H * (dv / bwd::kCols);
-  const size_t scr = ctas * bwd::kBlk * dk * bwd::kCols * sizeof(float);
+  const size_t scr = (size_t)n_seq * H * bwd::kBlk * dk * dv * sizeof(float);
   return (ck + 255) / 256 * 256 + (scr + 255) / 256 * 256;
 }
 
@@ -293,10 +302,20 @@ static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, con
                                 int gate, float* dq, float* dk, float* dv, float* dla,
                                 float* dbeta, float* d_init, float* ckpt, float* scratch,
                                 cudaStream_t stream) {
-  const long long blocks = (long long)n_seq * H * (DV / bwd::kCols);
-  bwd::backward_kernel<TIn, DK, DV><<<(unsigned)blocks, DK, 0, stream>>>(
-      (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, s0, cu, (const TIn*)d_o, d_final,
-      T, H, gate, dq, dk, dv, dla, dbeta, d_init, ckpt, scratch);
+  // Few chains: narrow slices, so that enough CTAs run to hide the per-token
+  // latency of each chain (2 x 148 CTAs of the wide slices fill a B200).
+  const long long chains = (long long)n_seq * H;
+  if (chains * (DV / bwd::kColsWide) < 2 * 148) {
+    constexpr int kC = bwd::kColsNarrow;
+    bwd::backward_kernel<TIn, DK, DV, kC><<<(unsigned)(chains * (DV / kC)), DK, 0, stream>>>(
+        (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, s0, cu, (const TIn*)d_o, d_final,
+        T, H, gate, dq, dk, dv, dla, dbeta, d_init, ckpt, scratch);
+  } else {
+    constexpr int kC = bwd::kColsWide;
+    bwd::backward_kernel<TIn, DK, DV, kC><<<(unsigned)(chains * (DV / kC)), DK, 0, stream>>>(
+        (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, s0, cu, (const TIn*)d_o, d_final,
+        T, H, gate, dq, dk, dv, dla, dbeta, d_init, ckpt, scratch);
+  }
   return cudaGetLastError();
 }
 

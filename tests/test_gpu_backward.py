@@ -94,3 +94,8 @@ def test_backward_packed_sequences():
 
 def test_backward_long_sequence_many_blocks():
     _check(_case(1, 700, 2, 128, 128, torch.float32, "channel", seed=11), "channel")
+
+
+def test_backward_many_chains_wide_slices():
+    # enough chains that each CTA takes 32 value columns (few chains take 8)
+    _check(_case(2, 40, 80, 128, 128, torch.float32, "channel", seed=13), "channel")
