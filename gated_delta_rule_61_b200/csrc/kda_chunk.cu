@@ -1123,19 +1123,8 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       tc::mma_commit(mbar);
       pend_mma = true;
     }
-    if (kRing <= 2 && n + step < n_chunks) {   // next own chunk, while the MMAs run
-      if (!gates(chunk_len(n + step))) {
-        ok = false;
-        break;
-      }
-    }
-    ok = cta_wait(mbar, phase, 3);
-    if (!ok) break;
-    pend_mma = false;
-    phase ^= 1;
-
     // ---- P8: S^T += D^T K~ (tf32, A from TMEM, B K-major); O^T += D^T M_qk^T
-    if (tid == 0) {
+    auto issue_update = [&]() {
       constexpr uint32_t id_s = tc::make_idesc(2, 0, 0, 128, 128);
       constexpr uint32_t id_o = tc::make_idesc(2, 0, 0, 128, 64);
       const uint64_t dk0 = tc::make_desc(sbase + OFF_KT, 16, 1024);
@@ -1149,7 +1138,36 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         tc::mma_tf32_ts(tmem + TM_O, a_t, dm, id_o, 1u);
       }
       tc::mma_commit(mbar);
-      pend_mma = true;
+    };
+    if constexpr (kRing > 2) {
+      // On the ring's critical path: only the issuing thread needs the D/O
+      // results before the update's MMAs, so it waits for them alone and
+      // issues the update at once; one CTA barrier afterwards shares the
+      // outcome. (With one or two CTAs per chain the gate scan runs here and
+      // its barriers wait for the issuing warp anyway.)
+      int fail7 = 0;
+      if (tid == 0) {
+        if (tc::mbar_wait_bounded(mbar, phase, kMaxWaitNs)) {
+          tc::fence_after_sync();
+          issue_update();
+        } else {
+          fail7 = 1;
+        }
+      }
+      fail7 = __syncthreads_or(fail7);
+      if (fail7) {   // the D/O MMAs are still pending (phase unchanged)
+        if (tid == 0) report_timeout(3);
+        ok = false;
+        break;
+      }
+      phase ^= 1;   // the D/O MMAs completed; the update's commit is the next phase
+    } else {
+      if (n + step < n_chunks)   // next own chunk, while the MMAs run
+        gates(chunk_len(n + step));
+      ok = cta_wait(mbar, phase, 3);
+      if (!ok) break;
+      phase ^= 1;
+      if (tid == 0) issue_update();
     }
     {
       const bool next = n + step < n_chunks;   // its k and v were issued at P5
