@@ -190,7 +190,8 @@ decode_multi_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
   const int col = slice * CW + 4 * cg;
   const bool raw_qk = flags & kRawQK;
 
-  __shared__ float s_k[kMaxT][DK], s_q[kMaxT][DK], s_a[kMaxT][DK];
+  // per token and key row: {decay, k, q, unused}, one 16-byte load per row
+  __shared__ float4 s_akq[kMaxT][DK];
   __shared__ __align__(16) float s_v[kMaxT][CW];
   __shared__ float s_beta[kMaxT], s_kq[kMaxT], s_ik[kMaxT], s_iq[kMaxT];
   __shared__ float4 s_red[2][kWarps][2][LPR];
@@ -221,12 +222,10 @@ decode_multi_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
         nk = fmaf(kk, kk, nk);
         nq = fmaf(qq, qq, nq);
       }
-      s_k[t][i] = kk;
-      s_q[t][i] = qq;
       float a = 1.f;
       if (gate == kGateChannel) a = decay_from(__ldg(log_alpha + tok * DK + i), flags);
       else if (gate == kGateScalar) a = decay_from(__ldg(log_alpha + tok), flags);
-      s_a[t][i] = a;
+      s_akq[t][i] = make_float4(a, kk, qq, 0.f);
       kqg[g] = kk * qq;
     }
     for (int j = lane; j < CW; j += 32) s_v[t][j] = Io<TIn>::load(v + tok * DV + slice * CW + j);
@@ -260,7 +259,8 @@ decode_multi_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
 #pragma unroll
     for (int i = 0; i < NI; ++i) {
       const int row = (warp + i * kWarps) * RPI + sub;
-      const float a = s_a[t][row], kk = s_k[t][row], qq = s_q[t][row];
+      const float4 akq = s_akq[t][row];
+      const float a = akq.x, kk = akq.y, qq = akq.z;
       s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
       r.x = fmaf(s[i].x, kk, r.x); r.y = fmaf(s[i].y, kk, r.y);
       r.z = fmaf(s[i].z, kk, r.z); r.w = fmaf(s[i].w, kk, r.w);
@@ -301,7 +301,7 @@ decode_multi_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
 #pragma unroll
     for (int i = 0; i < NI; ++i) {
       const int row = (warp + i * kWarps) * RPI + sub;
-      const float kk = s_k[t][row] * ik;
+      const float kk = s_akq[t][row].y * ik;
       s[i].x = fmaf(kk, d[0], s[i].x); s[i].y = fmaf(kk, d[1], s[i].y);
       s[i].z = fmaf(kk, d[2], s[i].z); s[i].w = fmaf(kk, d[3], s[i].w);
     }
