@@ -168,8 +168,9 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
 // the same state pass, with all T tokens' inputs staged into shared memory
 // first (k, q and the decay per key row after the prologue; v of this CTA's
 // columns; beta, k.q and the normalisation scales per token), which also
-// overlaps those loads with the state loads. The token loop then needs one
-// CTA barrier per token (the cross-warp part of r and p, double-buffered).
+// overlaps those loads with the state loads. The token loop then needs two
+// CTA barriers per token (the cross-warp part of r and p is added once per
+// value, not by every warp; double-buffered).
 template <typename TIn, int DK, int DV, int SPLIT>
 __global__ void __launch_bounds__(256, decode_min_blocks<SPLIT>())
 decode_multi_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
@@ -195,6 +196,7 @@ decode_multi_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
   __shared__ __align__(16) float s_v[kMaxT][CW];
   __shared__ float s_beta[kMaxT], s_kq[kMaxT], s_ik[kMaxT], s_iq[kMaxT];
   __shared__ float4 s_red[2][kWarps][2][LPR];
+  __shared__ __align__(16) float s_fin[2][2][4 * LPR];   // r and p of the CTA's columns
 
   float* S = state + (size_t)head * DK * DV;
   float4 s[NI];
@@ -279,14 +281,19 @@ decode_multi_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
       s_red[buf][warp][1][cg] = p;
     }
     __syncthreads();
-    r = make_float4(0.f, 0.f, 0.f, 0.f);
-    p = r;
+    // The warps' partial sums, added once per value (in warp order, as the
+    // plain step does) by the first 8 LPR threads, then read by all.
+    if (threadIdx.x < 8 * LPR) {
+      const int rp = threadIdx.x / (4 * LPR), cc = threadIdx.x % (4 * LPR);
+      const float* part = reinterpret_cast<const float*>(&s_red[buf][0][rp][0]) + cc;
+      float acc = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      const float4 x = s_red[buf][w][0][cg], y = s_red[buf][w][1][cg];
-      r.x += x.x; r.y += x.y; r.z += x.z; r.w += x.w;
-      p.x += y.x; p.y += y.y; p.z += y.z; p.w += y.w;
+      for (int w = 0; w < kWarps; ++w) acc += part[w * 8 * LPR];
+      s_fin[buf][rp][cc] = acc;
     }
+    __syncthreads();
+    r = *reinterpret_cast<const float4*>(&s_fin[buf][0][4 * cg]);
+    p = *reinterpret_cast<const float4*>(&s_fin[buf][1][4 * cg]);
     const float ik = s_ik[t], iq = s_iq[t], kq = s_kq[t], bb = s_beta[t];
     const float4 vv = *reinterpret_cast<const float4*>(&s_v[t][4 * cg]);
     const float d[4] = {bb * (vv.x - r.x * ik), bb * (vv.y - r.y * ik), bb * (vv.z - r.z * ik),
