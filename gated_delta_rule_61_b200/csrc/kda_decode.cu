@@ -19,8 +19,8 @@
 // own v entries); 256 threads = 8 warps; every lane streams 128-bit vectors of
 // whole contiguous rows, holds its rows in registers for the whole call, and
 // the two column reductions go through shuffles and one small shared-memory
-// exchange per token. Two kernels: the plain decode step, and the general one
-// (several tokens, gate forms, prologue).
+// exchange per token. Two kernels: the single step (any gate form and
+// prologue; the plain form compiled on its own), and the several-token one.
 #include "kda_common.cuh"
 
 namespace kda {
@@ -38,7 +38,8 @@ __device__ __forceinline__ float decay_from(float g, unsigned flags) {
   return (flags & kRawGate) ? sigmoid_f(g) : expf(g);
 }
 
-// The plain decode step (one token, per-channel gate, ready inputs).
+// The decode step (one token; any gate form; the prologue flags applied to
+// the small per-head vectors).
 // CTA (head, slice) owns value columns [slice * DV / SPLIT, +DV / SPLIT).
 // Within a CTA each lane owns one 4-column group; LPR = columns / 4 lanes
 // cover a row, so a warp instruction reads RPI = 32 / LPR whole rows (512
@@ -47,14 +48,18 @@ __device__ __forceinline__ float decay_from(float g, unsigned flags) {
 template <int SPLIT>
 constexpr int decode_min_blocks() { return SPLIT == 1 ? 2 : 4; }
 
-template <typename TIn, int DK, int DV, int SPLIT>
+// kForms: the gate form and prologue flags are read (gate, flags); without
+// it the kernel is the plain step (per-channel gate, ready inputs).
+template <typename TIn, int DK, int DV, int SPLIT, bool kForms>
 __global__ void __launch_bounds__(256, decode_min_blocks<SPLIT>())
 decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
                    const TIn* __restrict__ v, const float* __restrict__ log_alpha,
                    const float* __restrict__ beta, float* __restrict__ state,
-                   TIn* __restrict__ o) {
+                   TIn* __restrict__ o, int gate_arg, unsigned flags_arg) {
   constexpr int kWarps = 8;
   constexpr int CW = DV / SPLIT;          // value columns of this CTA
+  const int gate = kForms ? gate_arg : kGateChannel;
+  const unsigned flags = kForms ? flags_arg : 0u;
   constexpr int LPR = CW / 4;             // lanes per row (one float4 each)
   constexpr int RPI = 32 / LPR;           // rows per warp instruction
   constexpr int NI = DK / (kWarps * RPI); // float4 per thread
@@ -67,7 +72,8 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
 
   __shared__ float s_k[DK], s_q[DK], s_a[DK];
   __shared__ float4 s_red[kWarps][2][LPR];
-  __shared__ float s_kq[kWarps];
+  __shared__ float s_kq[kWarps], s_nk[kWarps], s_nq[kWarps];
+  const bool raw_qk = flags & kRawQK;
 
   float* S = state + (size_t)head * DK * DV;
 
@@ -88,20 +94,40 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
   if (threadIdx.x < DK) {
     kk0 = Io<TIn>::load(k + (size_t)head * DK + threadIdx.x);
     qq0 = Io<TIn>::load(q + (size_t)head * DK + threadIdx.x);
-    la0 = __ldg(log_alpha + (size_t)head * DK + threadIdx.x);
+    if (gate == kGateChannel) la0 = __ldg(log_alpha + (size_t)head * DK + threadIdx.x);
+    else if (gate == kGateScalar) la0 = __ldg(log_alpha + head);
   }
 
-  // Small per-head vectors: k, q, alpha = exp(log_alpha); k . q per warp.
-  float kq_part = 0.f;
+  // Small per-head vectors: k, q (SiLU of raw projections; their norms are
+  // applied as scales below), the decay alpha; k . q (and the squared norms)
+  // per warp.
+  float kq_part = 0.f, nk_part = 0.f, nq_part = 0.f;
   if (threadIdx.x < DK) {
+    if (raw_qk) {
+      kk0 = silu_f(kk0);
+      qq0 = silu_f(qq0);
+      nk_part = kk0 * kk0;
+      nq_part = qq0 * qq0;
+    }
     s_k[threadIdx.x] = kk0;
     s_q[threadIdx.x] = qq0;
-    s_a[threadIdx.x] = expf(la0);
+    s_a[threadIdx.x] = gate == kGateNone ? 1.f : decay_from(la0, flags);
     kq_part = kk0 * qq0;
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) kq_part += __shfl_xor_sync(0xffffffffu, kq_part, off);
-  if (lane == 0) s_kq[warp] = kq_part;
+  if (raw_qk) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      nk_part += __shfl_xor_sync(0xffffffffu, nk_part, off);
+      nq_part += __shfl_xor_sync(0xffffffffu, nq_part, off);
+    }
+  }
+  if (lane == 0) {
+    s_kq[warp] = kq_part;
+    s_nk[warp] = nk_part;
+    s_nq[warp] = nq_part;
+  }
   __syncthreads();
 
   // Decay rows and accumulate partial r = S'^T k and p = S'^T q.
@@ -140,21 +166,36 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
     r.x += a.x; r.y += a.y; r.z += a.z; r.w += a.w;
     p.x += b.x; p.y += b.y; p.z += b.z; p.w += b.w;
   }
-  const float bb = __ldg(beta + head);
+  // L2 normalisation of SiLU(k), SiLU(q) (x / max(|x|, 1e-12)) as scales of
+  // r, p, k . q and k (exactly 1 without the prologue)
+  float ik = 1.f, iq = 1.f;
+  if (raw_qk) {
+    float nk = 0.f, nq = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      nk += s_nk[w];
+      nq += s_nq[w];
+    }
+    ik = 1.f / fmaxf(sqrtf(nk), 1e-12f);
+    iq = 1.f / fmaxf(sqrtf(nq), 1e-12f);
+    kq = kq * ik * iq;
+  }
+  float bb = __ldg(beta + head);
+  if (flags & kRawBeta) bb = sigmoid_f(bb);
   const float rr[4] = {r.x, r.y, r.z, r.w}, pp[4] = {p.x, p.y, p.z, p.w};
   float d[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    d[j] = bb * (Io<TIn>::load(v + (size_t)head * DV + col + j) - rr[j]);
+    d[j] = bb * (Io<TIn>::load(v + (size_t)head * DV + col + j) - rr[j] * ik);
     if (warp == 0 && sub == 0)
-      Io<TIn>::store(o + (size_t)head * DV + col + j, fmaf(kq, d[j], pp[j]));
+      Io<TIn>::store(o + (size_t)head * DV + col + j, fmaf(kq, d[j], pp[j] * iq));
   }
 
   // S = S' + k d^T, written once.
 #pragma unroll
   for (int i = 0; i < NI; ++i) {
     const int row = (warp + i * kWarps) * RPI + sub;
-    const float kk = s_k[row];
+    const float kk = s_k[row] * ik;
     s[i].x = fmaf(kk, d[0], s[i].x); s[i].y = fmaf(kk, d[1], s[i].y);
     s[i].z = fmaf(kk, d[2], s[i].z); s[i].w = fmaf(kk, d[3], s[i].w);
     __stcs(reinterpret_cast<float4*>(S + (size_t)row * DV + col), s[i]);
@@ -164,7 +205,7 @@ decode_step_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// Every other decode call (1 to 16 tokens, any gate form, prologue flags):
+// Calls with 2 to 16 tokens (any gate form, prologue flags):
 // the same state pass, with all T tokens' inputs staged into shared memory
 // first (k, q and the decay per key row after the prologue; v of this CTA's
 // columns; beta, k.q and the normalisation scales per token), which also
@@ -325,7 +366,8 @@ static cudaError_t launch_decode_split(const void* q, const void* k, const void*
                                        const float* la, const float* beta, float* state,
                                        void* o, int n_heads, int T, int H, int gate,
                                        unsigned flags, cudaStream_t stream) {
-  if (T == 1 && gate == kGateChannel && flags == 0u) {
+  if (T == 1) {
+    const bool forms = gate != kGateChannel || flags != 0u;
     // programmatic dependent launch: scheduled while the previous kernel on
     // the stream finishes (the kernel waits for it before reading anything)
     cudaLaunchConfig_t cfg = {};
@@ -337,8 +379,13 @@ static cudaError_t launch_decode_split(const void* q, const void* k, const void*
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_step_kernel<TIn, DK, DV, kSplit>, (const TIn*)q,
-                              (const TIn*)k, (const TIn*)v, la, beta, state, (TIn*)o);
+    if (forms)
+      return cudaLaunchKernelEx(&cfg, decode_step_kernel<TIn, DK, DV, kSplit, true>,
+                                (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, state,
+                                (TIn*)o, gate, flags);
+    return cudaLaunchKernelEx(&cfg, decode_step_kernel<TIn, DK, DV, kSplit, false>,
+                              (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, state,
+                              (TIn*)o, gate, flags);
   }
   decode_multi_kernel<TIn, DK, DV, kSplit><<<n_heads * kSplit, 256, 0, stream>>>(
       (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, state, (TIn*)o, T, H, gate, flags);
