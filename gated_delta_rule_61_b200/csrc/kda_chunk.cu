@@ -566,6 +566,7 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
   float2 lr[8];
   uint32_t qr[8];
   float bt[2];   // warp 0 only: beta of rows 2 lane, 2 lane + 1
+  float gt[2];   // warp 0 only, one decay per token: log_alpha of the same rows
   auto chunk_len = [&](int nn) {
     const long long tc0 = t_begin + (long long)nn * C;
     return (int)((t_end - tc0) < C ? (t_end - tc0) : C);
@@ -591,19 +592,19 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       qr[i] = 0u;
       if (r < Lc) {
         const size_t tok = (size_t)(tc0 + r) * H + head;
-        if constexpr (kGate == 0) {
-          lr[i] = ld_stream_f2(log_alpha + tok * DK + c0);
-        } else if constexpr (kGate == 1) {
-          const float x = __ldg(log_alpha + tok);
-          lr[i] = make_float2(x, x);
-        }
+        if constexpr (kGate == 0) lr[i] = ld_stream_f2(log_alpha + tok * DK + c0);
         qr[i] = ld_stream_u32(q + tok * DK + c0);
       }
     }
     bt[0] = bt[1] = 0.f;
+    gt[0] = gt[1] = 0.f;
     if (warp == 0) {
       if (2 * lane < Lc) bt[0] = __ldg(beta + (size_t)(tc0 + 2 * lane) * H + head);
       if (2 * lane + 1 < Lc) bt[1] = __ldg(beta + (size_t)(tc0 + 2 * lane + 1) * H + head);
+      if constexpr (kGate == 1) {
+        if (2 * lane < Lc) gt[0] = __ldg(log_alpha + (size_t)(tc0 + 2 * lane) * H + head);
+        if (2 * lane + 1 < Lc) gt[1] = __ldg(log_alpha + (size_t)(tc0 + 2 * lane + 1) * H + head);
+      }
     }
   };
   if (rank < n_chunks) {
@@ -618,6 +619,68 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
   // D/O MMA is in flight; it touches no operand tile.
   float g0[8], g1[8];
   auto gates = [&](int Lc) -> bool {
+    if constexpr (kGate == 2) {
+      // No decay: only beta is published (and a unit chunk decay).
+      if (warp == 0) {
+        float b0 = bt[0], b1 = bt[1];
+        if (flags & 2u) {
+          b0 = 2 * lane < Lc ? sigmoid_fast(b0) : 0.f;
+          b1 = 2 * lane + 1 < Lc ? sigmoid_fast(b1) : 0.f;
+        }
+        *reinterpret_cast<float2*>(s_beta + 2 * lane) = make_float2(b0, b1);
+      }
+      if (tid < 128) s_gamma[tid] = 1.f;
+      __syncthreads();
+      return true;
+    }
+    if constexpr (kGate == 1) {
+      // One decay per token: warp 0 scans the chunk's 64 values (lane l holds
+      // rows 2 l and 2 l + 1, i.e. sub-chunk l / 8, pair l % 8) into the
+      // cumulative gate per row, summing in the per-channel scan's order (pair
+      // sums, exclusive sum over the sub-chunk's pairs, then the sub-chunk
+      // totals), so both forms give the same bits for the same decays.
+      if (warp == 0) {
+        float b0 = bt[0], b1 = bt[1];
+        if (flags & 2u) {
+          b0 = 2 * lane < Lc ? sigmoid_fast(b0) : 0.f;
+          b1 = 2 * lane + 1 < Lc ? sigmoid_fast(b1) : 0.f;
+        }
+        *reinterpret_cast<float2*>(s_beta + 2 * lane) = make_float2(b0, b1);
+        float x0 = gt[0], x1 = gt[1];
+        if (flags & 4u) {
+          if (2 * lane < Lc) x0 = log_sigmoid_fast(x0);
+          if (2 * lane + 1 < Lc) x1 = log_sigmoid_fast(x1);
+        }
+        x0 = fmaxf(x0, kLogAlphaMin);
+        x1 = fmaxf(x1, kLogAlphaMin);
+        const float pr = x0 + x1;
+        const int grp0 = lane & ~7, pos = lane & 7;
+        float run = 0.f, excl = 0.f;
+#pragma unroll
+        for (int r8 = 0; r8 < 8; ++r8) {
+          const float x = __shfl_sync(0xffffffffu, pr, grp0 + r8);
+          if (r8 == pos) excl = run;
+          run += x;
+        }
+        const float t0 = __shfl_sync(0xffffffffu, run, 0);
+        const float t1 = __shfl_sync(0xffffffffu, run, 8);
+        const float t2 = __shfl_sync(0xffffffffu, run, 16);
+        const float tb1 = t0, tb2 = tb1 + t1, tb3 = tb2 + t2;
+        const int a = lane >> 3;
+        const float tb = a == 0 ? 0.f : a == 1 ? tb1 : a == 2 ? tb2 : tb3;
+        const float ge = (tb + excl) + x0;
+        const float go = ge + x1;
+        *reinterpret_cast<float2*>(s_gf + 2 * lane) = make_float2(ge, go);   // per row
+        if (lane == 31) {
+          const float gam = __expf(go);   // decay over the whole chunk
+#pragma unroll
+          for (int c = 0; c < 128; c += 4)
+            *reinterpret_cast<float4*>(s_gamma + c) = make_float4(gam, gam, gam, gam);
+        }
+      }
+      __syncthreads();
+      return true;
+    }
     {
       float l0[8], l1[8];
       const bool raw_gate = kGate != 2 && (flags & 4u);
@@ -763,25 +826,36 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
       // Sub-chunk midpoints m_a and the per-channel factors, from five
       // exponentials per channel: e^{m_0}, e^{m_a - m_(a-1)} and e^{g_last - m_3};
       // every other factor is a product of these (all at most 1).
+      // Without decay every factor is 1 and no exponential is taken.
+      constexpr bool kDecay = kGate != 2;
+      auto ex = [](float x) { return kDecay ? __expf(x) : 1.f; };
       float mid0[4], mid1[4];
+      float gl0, gl1;
+      if constexpr (kGate == 1) {   // the per-row scan, the same on every channel
 #pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        mid0[a] = 0.5f * (s_gf[a * 128 + c0] + s_gl[a * 128 + c0]);
-        mid1[a] = 0.5f * (s_gf[a * 128 + c0 + 1] + s_gl[a * 128 + c0 + 1]);
+        for (int a = 0; a < 4; ++a) mid0[a] = mid1[a] = 0.5f * (s_gf[16 * a] + s_gf[16 * a + 15]);
+        gl0 = gl1 = s_gf[63];
+      } else {
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          mid0[a] = kDecay ? 0.5f * (s_gf[a * 128 + c0] + s_gl[a * 128 + c0]) : 0.f;
+          mid1[a] = kDecay ? 0.5f * (s_gf[a * 128 + c0 + 1] + s_gl[a * 128 + c0 + 1]) : 0.f;
+        }
+        gl0 = kDecay ? s_gl[3 * 128 + c0] : 0.f;
+        gl1 = kDecay ? s_gl[3 * 128 + c0 + 1] : 0.f;
       }
-      const float gl0 = s_gl[3 * 128 + c0], gl1 = s_gl[3 * 128 + c0 + 1];
       float dd0[4], dd1[4];   // dd[a] = e^{m_a - m_(a-1)}, a >= 1
       dd0[0] = dd1[0] = 1.f;
 #pragma unroll
       for (int a = 1; a < 4; ++a) {
-        dd0[a] = __expf(mid0[a] - mid0[a - 1]);
-        dd1[a] = __expf(mid1[a] - mid1[a - 1]);
+        dd0[a] = ex(mid0[a] - mid0[a - 1]);
+        dd1[a] = ex(mid1[a] - mid1[a - 1]);
       }
       float em0[4], em1[4], kt0[4], kt1[4];
-      em0[0] = __expf(mid0[0]);
-      em1[0] = __expf(mid1[0]);
-      kt0[3] = __expf(gl0 - mid0[3]);
-      kt1[3] = __expf(gl1 - mid1[3]);
+      em0[0] = ex(mid0[0]);
+      em1[0] = ex(mid1[0]);
+      kt0[3] = ex(gl0 - mid0[3]);
+      kt1[3] = ex(gl1 - mid1[3]);
 #pragma unroll
       for (int a = 1; a < 4; ++a) {
         em0[a] = em0[a - 1] * dd0[a];
@@ -834,8 +908,12 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
           q0 = silu_tanh(q0) * iq;
           q1 = silu_tanh(q1) * iq;
         }
-        const float f0 = __expf(g0[i] - mid0[a]), f1 = __expf(g1[i] - mid1[a]);
-        const float fi0 = rcp_approx(f0), fi1 = rcp_approx(f1);
+        // this row's cumulative gate per channel (per row with one decay per token)
+        const float gi0 = kGate == 1 ? s_gf[16 * a + 2 * rg + e] : g0[i];
+        const float gi1 = kGate == 1 ? gi0 : g1[i];
+        const float f0 = kDecay ? __expf(gi0 - mid0[a]) : 1.f;
+        const float f1 = kDecay ? __expf(gi1 - mid1[a]) : 1.f;
+        const float fi0 = kDecay ? rcp_approx(f0) : 1.f, fi1 = kDecay ? rcp_approx(f1) : 1.f;
         *reinterpret_cast<uint32_t*>(pAGk + ro) = pack_bf16x2(k0 * f0, k1 * f1);
         *reinterpret_cast<uint32_t*>(pAGk + ro + 8192) = pack_bf16x2(q0 * f0, q1 * f1);
         const float e0 = k0 * fi0, e1 = k1 * fi1;
@@ -847,8 +925,8 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         // product is still representable (starting from E_j, which can be
         // e^75, lost terms of size e^{g_r - g_j} under strong decay).
         if (a < 3) {
-          float n0 = k0 * __expf(mid0[a < 3 ? a + 1 : 3] - g0[i]);
-          float n1 = k1 * __expf(mid1[a < 3 ? a + 1 : 3] - g1[i]);
+          float n0 = kDecay ? k0 * __expf(mid0[a < 3 ? a + 1 : 3] - gi0) : k0;
+          float n1 = kDecay ? k1 * __expf(mid1[a < 3 ? a + 1 : 3] - gi1) : k1;
           const uint32_t set_off = a == 0 ? 8192u : a == 1 ? 10240u : 14336u;
           *reinterpret_cast<uint32_t*>(pBGe + ro + set_off) = pack_bf16x2(n0, n1);
           if (a < 2) {
