@@ -137,7 +137,7 @@ def test_scalar_gate_equals_broadcast_channel_gate_on_the_gpu():
 # Decode: T tokens per call against the cached state
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("T", [1, 2, 4, 16])
+@pytest.mark.parametrize("T", [1, 2, 4, 7, 16])
 @pytest.mark.parametrize("gate", ["channel", "scalar", "none"])
 @pytest.mark.parametrize("raw", [False, True])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
@@ -155,6 +155,43 @@ def test_multi_token_decode_against_oracle(T, gate, raw, dtype):
     tol_o = TOL_F32 if dtype == torch.float32 else TOL_BF16_O
     assert_close(o, o_ref, tol_o, "decode T=%d o" % T)
     assert_close(S, s_ref, TOL_F32, "decode T=%d state" % T)
+
+
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (128, 64), (64, 128)])
+@pytest.mark.parametrize("B,H", [(3, 2), (40, 4)])
+def test_multi_token_decode_head_shapes(dk, dv, B, H):
+    """Every head shape, with few heads (16-column slices) and with enough
+    heads for the wide slices."""
+    T = 6
+    inp = _inputs(B, T, H, dk, dv, torch.bfloat16, "channel", False, seed=7 + dk + dv + B,
+                  init_std=None)
+    S0 = decode_state(B, H, dk, dv, std=0.05, seed=B + dv)
+    inp["init_state"] = S0
+    o_ref, s_ref = _oracle(inp, "channel", False, clamp=False)
+    g = {n: (x.cuda() if isinstance(x, torch.Tensor) else x) for n, x in inp.items()}
+    S = S0.cuda()
+    o = kda.decode(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], S)
+    torch.cuda.synchronize()
+    assert_close(o, o_ref, TOL_BF16_O, "decode head shape o")
+    assert_close(S, s_ref, TOL_F32, "decode head shape state")
+
+
+@pytest.mark.parametrize("gate", ["channel", "scalar"])
+def test_multi_token_decode_full_gate_inside_a_chunk(gate):
+    """log_alpha = -inf at the third of seven tokens clears the state there
+    (a decay of exactly zero inside a call)."""
+    B, T, H, d = 2, 7, 3, 128
+    inp = _inputs(B, T, H, d, d, torch.float32, gate, False, seed=91, init_std=None)
+    inp["log_alpha"][:, 2] = -float("inf")
+    S0 = decode_state(B, H, d, d, std=0.05, seed=9)
+    inp["init_state"] = S0
+    o_ref, s_ref = _oracle(inp, gate, False, clamp=False)
+    g = {n: (x.cuda() if isinstance(x, torch.Tensor) else x) for n, x in inp.items()}
+    S = S0.cuda()
+    o = kda.decode(g["q"], g["k"], g["v"], g["log_alpha"], g["beta"], S, gate=gate)
+    torch.cuda.synchronize()
+    assert_close(o, o_ref, TOL_F32, "decode full gate o")
+    assert_close(S, s_ref, TOL_F32, "decode full gate state")
 
 
 @pytest.mark.parametrize("T", [2, 7, 16])
