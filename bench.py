@@ -263,6 +263,40 @@ def _time_calls(fn, n, stream):
     return a.elapsed_time(b) / n
 
 
+def bench_backward(args, dev, stream, hbm, world, inp):
+    """Backward of the prefill workload (gradients of every input and the
+    initial state from dL/do and dL/dS_final); --backward-tokens takes the
+    first N tokens of each sequence instead of all of them."""
+    import torch
+    from gated_delta_rule_61_b200 import kda
+    P = PREFILL
+    T = args.backward_tokens or P["T"]
+    x = {n: inp[n][:, :T].contiguous() for n in ("q", "k", "v", "log_alpha", "beta")}
+    x["init_state"] = inp["init_state"]
+    head_tokens = P["B"] * T * P["H"]
+    state_bytes = 2 * P["B"] * P["H"] * P["dk"] * P["dv"] * 4
+    g = torch.Generator(device=dev).manual_seed(78)
+    d_o = torch.randn(x["v"].shape, device=dev, generator=g).to(x["v"].dtype)
+    d_fin = torch.randn(x["init_state"].shape, device=dev, generator=g)
+    need = kda.lib().kda_backward_workspace_bytes(P["B"], P["B"] * T, P["H"], P["dk"], P["dv"])
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    ms = _time_calls(lambda: kda.backward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"],
+                                          d_o, init_state=x["init_state"], d_final=d_fin,
+                                          workspace=ws, stream=stream), 2, stream)
+    # bytes: the forward inputs read twice (checkpoint pass and block
+    # recomputation), d_o, the fp32 gradients written, states
+    per = 2 * (3 * 256 + 512 + 4) + 256 + 4 * (3 * 128 + 128 + 1)
+    gbs = (head_tokens * per + 3 * state_bytes) / (ms * 1e-3) / 1e9
+    out = {"workload": "KDA backward of B=%d T=%d H=%d d=128 bf16 (token-recurrent, "
+                       "checkpoints every 16 tokens)" % (P["B"], T, P["H"]),
+           "ms_per_call": ms, "tokens_per_s": world * P["B"] * T / (ms * 1e-3),
+           "roofline": {"bound": "latency (serial token chain)", "achieved": gbs,
+                        "peak": hbm, "unit": "GB/s", "frac": gbs / hbm}}
+    del d_o, d_fin, ws, x
+    torch.cuda.empty_cache()
+    return out
+
+
 def bench_forms(args, dev, stream, hbm, world, inp, dec):
     """The other gate forms (one decay per token, none), the fused input
     prologue (raw q/k projections, beta and gate logits) and multi-token
@@ -355,29 +389,6 @@ def bench_forms(args, dev, stream, hbm, world, inp, dec):
     out["decode_multi_token"] = {
         "workload": "B=256 H=32 d=128, T tokens per sequence per call, state in place",
         **multi}
-    # backward of the prefill workload (gradients of every input and the
-    # initial state from dL/do and dL/dS_final)
-    if not args.no_backward:
-        d_o = torch.randn(inp["v"].shape, device=dev, generator=g).to(inp["v"].dtype)
-        d_fin = torch.randn(inp["init_state"].shape, device=dev, generator=g)
-        need = kda.lib().kda_backward_workspace_bytes(P["B"], P["B"] * P["T"], P["H"], P["dk"],
-                                                      P["dv"])
-        ws = torch.empty(need, dtype=torch.uint8, device=dev)
-        ms = _time_calls(lambda: kda.backward(inp["q"], inp["k"], inp["v"], inp["log_alpha"],
-                                              inp["beta"], d_o, init_state=inp["init_state"],
-                                              d_final=d_fin, workspace=ws, stream=stream),
-                         2, stream)
-        # bytes: the forward inputs read twice (checkpoint pass and block
-        # recomputation), d_o, the fp32 gradients written, states
-        per = 2 * (3 * 256 + 512 + 4) + 256 + 4 * (3 * 128 + 128 + 1)
-        gbs = (head_tokens * per + 3 * state_bytes) / (ms * 1e-3) / 1e9
-        out["backward"] = {
-            "workload": "KDA backward of B=4 T=8192 H=16 d=128 bf16 (token-recurrent, "
-                        "checkpoints every 16 tokens)",
-            "ms_per_call": ms, "tokens_per_s": world * P["B"] * P["T"] / (ms * 1e-3),
-            "roofline": {"bound": "latency (serial token chain)", "achieved": gbs,
-                         "peak": hbm, "unit": "GB/s", "frac": gbs / hbm}}
-        del d_o, d_fin, ws
     del S
     torch.cuda.empty_cache()
     return out
@@ -583,6 +594,9 @@ def bench_ours(args):
     forms = None
     if not args.no_forms:
         forms = bench_forms(args, dev, stream, hbm, world, inp, dec)
+    bwd = None
+    if not args.no_backward:
+        bwd = bench_backward(args, dev, stream, hbm, world, inp)
     clk.__exit__(None, None, None)
 
     # ---------------- end to end through the public API (host buffers) ----------------
@@ -672,7 +686,7 @@ def bench_ours(args):
                          "peak_kind": peak_kind, "kernel_ms": kernel_ms,
                          "tensor": {"achieved_tflops": tflops, "peak_tflops": bf16_tf,
                                     "frac": tflops / bf16_tf}},
-            "decode": dec, "varlen": var, "long": lng, "forms": forms, "e2e": e2e,
+            "decode": dec, "varlen": var, "long": lng, "forms": forms, "backward": bwd, "e2e": e2e,
             "cpu_baseline": cpu,
             "gpu_launches": args.steps, "clocks": clk.summary(),
         }
@@ -697,6 +711,8 @@ def main():
                     help="tokens of the long-context prefill (default: the full workload)")
     ap.add_argument("--no-forms", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--backward-tokens", type=int, default=0,
+                    help="backward over the first N tokens of each sequence (default: all)")
     ap.add_argument("--varlen-seqs", type=int, default=64,
                     help="packed sequences of the varlen workload (a smaller case for profiling)")
     ap.add_argument("--varlen-max", type=int, default=32768,
