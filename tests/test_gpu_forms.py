@@ -122,13 +122,32 @@ def test_recurrent_gate_forms_and_prologue(gate, raw, dtype, dk, dv):
     assert_close(s, s_ref, tol_s, "recurrent state")
 
 
-def test_scalar_gate_equals_broadcast_channel_gate_on_the_gpu():
+@pytest.mark.parametrize("strong", [False, True])
+def test_scalar_gate_equals_broadcast_channel_gate_on_the_gpu(strong):
     """The same decay on every channel through the channel form gives the
-    scalar form's result (same kernel arithmetic, bit for bit)."""
+    scalar form's result (same kernel arithmetic, bit for bit), also with
+    strong decays (uniform in [-30, 0], some -inf) that the clamp reaches."""
     inp = _inputs(2, 150, 3, 128, 128, torch.bfloat16, "scalar", False, seed=5)
+    if strong:
+        g = torch.Generator().manual_seed(55)
+        la = -30.0 * torch.rand(2, 150, 3, generator=g)
+        la[torch.rand(2, 150, 3, generator=g) < 0.05] = -float("inf")
+        inp["log_alpha"] = la.float()
     o1, s1 = _gpu(inp, "scalar", False, 64)
     inp2 = dict(inp)
     inp2["log_alpha"] = inp["log_alpha"][..., None].expand(2, 150, 3, 128).contiguous()
+    o2, s2 = _gpu(inp2, "channel", False, 64)
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
+def test_no_gate_equals_zero_channel_gate_on_the_gpu():
+    """No decay through the specialised form equals log_alpha = 0 on every
+    channel through the per-channel form, bit for bit (every factor is
+    exactly 1 there)."""
+    inp = _inputs(2, 150, 3, 128, 128, torch.bfloat16, "none", False, seed=6)
+    o1, s1 = _gpu(inp, "none", False, 64)
+    inp2 = dict(inp)
+    inp2["log_alpha"] = torch.zeros(2, 150, 3, 128)
     o2, s2 = _gpu(inp2, "channel", False, 64)
     assert torch.equal(o1, o2) and torch.equal(s1, s2)
 
