@@ -100,3 +100,22 @@ def test_packed_sequences_each_launch_shape(lengths, H):
     for i, n in enumerate(lengths):
         if n == 0:
             assert torch.equal(s[i].cpu(), inp["init_state"][i].float())
+
+
+def test_launch_shape_does_not_change_the_bits():
+    """Chains are independent and every shape runs the same per-chunk
+    arithmetic (the state crosses L2 as exact fp32), so the same chains give
+    the same bits whether they run with one CTA each (80 chains), in rings of
+    two (40 chains) or in rings of four (6 chains)."""
+    assert _ring_for(80) == 1 and _ring_for(40) == 2 and _ring_for(6) == 4
+    inp = prefill_inputs(2, 150, 40, 128, 128, dtype=torch.bfloat16, seed=88, init_std=0.1,
+                         device="cpu")
+    o80, s80 = _run(inp)
+    part = {n: (inp[n][:1].contiguous() if inp[n] is not None else None) for n in inp}
+    o40, s40 = _run(part)
+    part = {n: (inp[n][:, :, :3].contiguous() if n in ("q", "k", "v", "log_alpha", "beta")
+                else inp[n]) for n in inp}
+    part["init_state"] = inp["init_state"][:, :3].contiguous()
+    o6, s6 = _run(part)
+    assert torch.equal(o40, o80[:1]) and torch.equal(s40, s80[:1])
+    assert torch.equal(o6, o80[:, :, :3]) and torch.equal(s6, s80[:, :3])
