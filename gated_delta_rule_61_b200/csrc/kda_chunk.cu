@@ -925,8 +925,21 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         // product is still representable (starting from E_j, which can be
         // e^75, lost terms of size e^{g_r - g_j} under strong decay).
         if (a < 3) {
-          float n0 = kDecay ? k0 * __expf(mid0[a < 3 ? a + 1 : 3] - gi0) : k0;
-          float n1 = kDecay ? k1 * __expf(mid1[a < 3 ? a + 1 : 3] - gi1) : k1;
+          // e^{m_(a+1) - g_j} = e^{m_(a+1) - m_a} e^{m_a - g_j}: a product of two
+          // factors already at hand while the first (at most 1) is a normal
+          // float; where it is tiny (decays averaging below about -4 per token)
+          // the product could have lost it, and the exponential is taken.
+          const int an = a < 3 ? a + 1 : 3;
+          float n0 = k0, n1 = k1;
+          if constexpr (kDecay) {
+            if (dd0[an] > 1e-30f && dd1[an] > 1e-30f) {
+              n0 = k0 * (fi0 * dd0[an]);
+              n1 = k1 * (fi1 * dd1[an]);
+            } else {
+              n0 = k0 * __expf(mid0[an] - gi0);
+              n1 = k1 * __expf(mid1[an] - gi1);
+            }
+          }
           const uint32_t set_off = a == 0 ? 8192u : a == 1 ? 10240u : 14336u;
           *reinterpret_cast<uint32_t*>(pBGe + ro + set_off) = pack_bf16x2(n0, n1);
           if (a < 2) {
