@@ -611,12 +611,13 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     issue_kv(rank);
     load_rows(rank);
   }
-  // Cumulative gates of a chunk from its log_alpha rows (lr):
-  // pair sums per (sub-chunk, rg) -> one exclusive scan over the 32 pairs per
-  // channel -> each thread adds its own rows. Writes g0/g1 (registers), beta,
-  // the first and last g of every sub-chunk and the chunk's decay e^{g_last}
-  // to shared memory. Runs for the next chunk while the current chunk's
-  // D/O MMA is in flight; it touches no operand tile.
+  // Cumulative gates of a chunk from its log_alpha rows (lr), one decay per
+  // key channel: pair sums per (sub-chunk, rg) -> one exclusive scan over the
+  // 32 pairs per channel -> each thread adds its own rows. Writes g0/g1
+  // (registers), beta, the first and last g of every sub-chunk and the
+  // chunk's decay e^{g_last} to shared memory. The other gate forms take the
+  // two shorter branches at the top. Runs for the next chunk while the
+  // current chunk's D/O MMA is in flight; it touches no operand tile.
   float g0[8], g1[8];
   auto gates = [&](int Lc) -> bool {
     if constexpr (kGate == 2) {
@@ -683,14 +684,14 @@ chunk64_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     }
     {
       float l0[8], l1[8];
-      const bool raw_gate = kGate != 2 && (flags & 4u);
+      const bool raw_gate = flags & 4u;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int r = 16 * (i >> 1) + 2 * rg + (i & 1);
         float x0 = lr[i].x, x1 = lr[i].y;   // zero past the chunk's end: no decay
         if (raw_gate && r < Lc) {
           x0 = log_sigmoid_fast(x0);
-          x1 = kGate == 1 ? x0 : log_sigmoid_fast(x1);
+          x1 = log_sigmoid_fast(x1);
         }
         l0[i] = fmaxf(x0, kLogAlphaMin);
         l1[i] = fmaxf(x1, kLogAlphaMin);
