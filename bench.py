@@ -10,7 +10,11 @@ carries the decode-step workload (B=256 sequences, H=32, d=128, fp32 state
 state-update GB/s, the packed variable-length prefill (64 sequences of
 log-uniform length in [128, 32768], H=32) and the long-context workload (one
 T=1,048,576 H=32 prefill, then 512 single-sequence decode steps replayed
-from a CUDA graph), each with its roofline fraction.
+from a CUDA graph), each with its roofline fraction; the other gate forms,
+the fused input prologue and multi-token decode ("forms"); the backward of
+the prefill workload ("backward", --backward-tokens N for the first N tokens
+of each sequence); and the end-to-end step through the public API from
+pinned host buffers, steps pipelined over three streams ("e2e").
 
   python bench.py [--gpus N --steps K --warmup W]        # this library
   python bench.py --impl reference [...]                 # the fp64 CPU oracle
