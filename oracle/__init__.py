@@ -267,3 +267,60 @@ def kda_decode_step(q, k, v, log_alpha, beta, state):
     B = q.shape[0]
     cu = np.arange(B + 1, dtype=np.int64)
     return kda_forward(q, k, v, la, b, init_state=state, cu_seqlens=cu)
+
+
+def _prologue_qk_vjp(x, g, eps=1e-12):
+    """Vector-Jacobian product of prologue_qk at the raw projection x with the
+    cotangent g (both [..., d]): with s = sigmoid(x), u = x s (SiLU), r = ||u||
+    and n = u / max(r, eps), the normalisation's Jacobian is (I - n n^T) / r
+    when r > eps and I / eps otherwise, and SiLU's derivative is
+    s (1 + x (1 - s))."""
+    x, g = _f64(x), _f64(g)
+    s = sigmoid(x)
+    u = x * s
+    r = np.sqrt(np.sum(u * u, axis=-1, keepdims=True))
+    n = u / np.maximum(r, eps)
+    du = np.where(r > eps, (g - n * np.sum(n * g, axis=-1, keepdims=True)) / np.maximum(r, eps),
+                  g / eps)
+    return du * s * (1.0 + x * (1.0 - s))
+
+
+def kda_backward_ex(q, k, v, log_alpha, beta, d_o, init_state=None, d_final=None,
+                    cu_seqlens=None, *, gate="channel", raw_qk=False, raw_beta=False,
+                    raw_gate=False, n_threads=None):
+    """Reverse mode of kda_forward_ex: the gradients with respect to the inputs
+    as given (raw projections and logits when the prologue flags are set).
+
+    The prologue is applied in fp64 as in kda_forward_ex, kda_backward gives
+    the gradients with respect to the transformed inputs, and the chain rule
+    takes them back through the prologue's elementwise definitions:
+    dq, dk through _prologue_qk_vjp; dbeta times sigmoid'(x) = s (1 - s);
+    dlog_alpha (summed over the key channels for the scalar gate) times
+    d log sigmoid(x) / dx = sigmoid(-x). With gate "none", dlog_alpha is None.
+    """
+    q0, k0 = _f64(q), _f64(k)
+    qn, kn = (prologue_qk(q0), prologue_qk(k0)) if raw_qk else (q0, k0)
+    b0 = _f64(beta)
+    b = sigmoid(b0) if raw_beta else b0
+    la_in = None
+    la = None
+    if gate != "none":
+        la_in = _f64(log_alpha)
+        la = log_sigmoid(la_in) if raw_gate else la_in
+    la = expand_gate(la, gate, qn.shape[:-1], qn.shape[-1])
+    g = kda_backward(qn, kn, v, la, b, d_o, init_state=init_state, d_final=d_final,
+                     cu_seqlens=cu_seqlens, n_threads=n_threads)
+    if raw_qk:
+        g["dq"] = _prologue_qk_vjp(q0, g["dq"])
+        g["dk"] = _prologue_qk_vjp(k0, g["dk"])
+    if raw_beta:
+        s = sigmoid(b0)
+        g["dbeta"] = g["dbeta"] * s * (1.0 - s)
+    if gate == "none":
+        g["dlog_alpha"] = None
+    else:
+        if gate == "scalar":
+            g["dlog_alpha"] = g["dlog_alpha"].sum(-1)
+        if raw_gate:
+            g["dlog_alpha"] = g["dlog_alpha"] * sigmoid(-la_in)
+    return g

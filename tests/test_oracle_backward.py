@@ -104,3 +104,65 @@ def test_full_clear_cuts_the_gradient_to_the_past():
     for n in ("dq", "dk", "dv", "dbeta"):
         assert np.all(g[n][:3] == 0), n
     assert np.all(g["d_init"] == 0)
+
+
+@pytest.mark.parametrize("gate", ["channel", "scalar", "none"])
+def test_backward_through_the_prologue_matches_finite_differences(gate):
+    """Raw projections (q, k through SiLU and L2 normalisation, beta and gate
+    logits through sigmoid and log-sigmoid): oracle.kda_backward_ex against
+    central differences of oracle.kda_forward_ex with the same flags."""
+    rng = np.random.default_rng(300 + len(gate))
+    T, H, dk, dv = 5, 2, 5, 4
+    gshape = {"channel": (T, H, dk), "scalar": (T, H), "none": None}[gate]
+    inp = dict(q=rng.standard_normal((T, H, dk)), k=rng.standard_normal((T, H, dk)),
+               v=rng.standard_normal((T, H, dv)),
+               log_alpha=None if gshape is None else rng.standard_normal(gshape) + 1.0,
+               beta=rng.standard_normal((T, H)),
+               init_state=rng.standard_normal((1, H, dk, dv)))
+    Wo = rng.standard_normal((T, H, dv))
+    Ws = rng.standard_normal((1, H, dk, dv))
+    flags = dict(gate=gate, raw_qk=True, raw_beta=True, raw_gate=True)
+
+    def loss():
+        o, S = oracle.kda_forward_ex(inp["q"], inp["k"], inp["v"], inp["log_alpha"],
+                                     inp["beta"], init_state=inp["init_state"], **flags)
+        return float(np.sum(o * Wo) + np.sum(S * Ws))
+
+    g = oracle.kda_backward_ex(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], Wo,
+                               init_state=inp["init_state"], d_final=Ws, **flags)
+    names = {"q": "dq", "k": "dk", "v": "dv", "beta": "dbeta", "init_state": "d_init"}
+    if gate != "none":
+        names["log_alpha"] = "dlog_alpha"
+    else:
+        assert g["dlog_alpha"] is None
+    h = 1e-6
+    for name, gname in names.items():
+        x = inp[name]
+        num = np.zeros_like(x)
+        for idx in np.ndindex(*x.shape):
+            keep = x[idx]
+            x[idx] = keep + h
+            lp = loss()
+            x[idx] = keep - h
+            lm = loss()
+            x[idx] = keep
+            num[idx] = (lp - lm) / (2 * h)
+        np.testing.assert_allclose(g[gname], num, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+def test_backward_ex_without_prologue_is_the_plain_reverse_mode():
+    """No flags: kda_backward_ex is kda_backward on the expanded gate, with
+    the scalar gate's gradient summed over the key channels it was copied to."""
+    rng = np.random.default_rng(9)
+    T, H, dk, dv = 6, 2, 5, 4
+    q, k = _unit(rng.standard_normal((T, H, dk))), _unit(rng.standard_normal((T, H, dk)))
+    v = rng.standard_normal((T, H, dv))
+    la = -rng.uniform(0.0, 1.5, (T, H))
+    b = rng.uniform(0.1, 1.0, (T, H))
+    s0 = rng.standard_normal((1, H, dk, dv))
+    Wo = rng.standard_normal((T, H, dv))
+    g = oracle.kda_backward_ex(q, k, v, la, b, Wo, init_state=s0, gate="scalar")
+    ref = oracle.kda_backward(q, k, v, np.repeat(la[..., None], dk, -1), b, Wo, init_state=s0)
+    for n in ("dq", "dk", "dv", "dbeta", "d_init"):
+        np.testing.assert_array_equal(g[n], ref[n])
+    np.testing.assert_array_equal(g["dlog_alpha"], ref["dlog_alpha"].sum(-1))
