@@ -296,7 +296,18 @@ def bench_backward(args, dev, stream, hbm, world, inp):
            "ms_per_call": ms, "tokens_per_s": world * P["B"] * T / (ms * 1e-3),
            "roofline": {"bound": "latency (serial token chain)", "achieved": gbs,
                         "peak": hbm, "unit": "GB/s", "frac": gbs / hbm}}
-    del d_o, d_fin, ws, x
+    # the same through the input prologue (raw q/k projections, beta and gate
+    # logits; the gradients are with respect to those)
+    raw = {n: torch.randn(x[n].shape, device=dev, generator=g).to(x[n].dtype) for n in ("q", "k")}
+    raw["beta"] = torch.randn(x["beta"].shape, device=dev, generator=g)
+    raw["log_alpha"] = torch.randn(x["log_alpha"].shape, device=dev, generator=g) + 3.0
+    ms_raw = _time_calls(lambda: kda.backward(raw["q"], raw["k"], x["v"], raw["log_alpha"],
+                                              raw["beta"], d_o, init_state=x["init_state"],
+                                              d_final=d_fin, workspace=ws, raw_qk=True,
+                                              raw_beta=True, raw_gate=True, stream=stream),
+                         2, stream)
+    out["raw_inputs_ms_per_call"] = ms_raw
+    del d_o, d_fin, ws, x, raw
     torch.cuda.empty_cache()
     return out
 

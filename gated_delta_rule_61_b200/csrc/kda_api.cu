@@ -21,9 +21,9 @@ cudaError_t launch_chunk64(const void* q, const void* k, const void* v, const fl
 cudaError_t launch_backward(const void* q, const void* k, const void* v, const float* la,
                             const float* beta, const float* s0, const int32_t* cu,
                             const void* d_o, const float* d_final, int n_seq, int T, int H,
-                            int dk, int dv, bool bf16, int gate, long long tokens, float* dq,
-                            float* dkk, float* dvv, float* dla, float* dbeta, float* d_init,
-                            void* workspace, cudaStream_t stream);
+                            int dk, int dv, bool bf16, int gate, unsigned flags,
+                            long long tokens, float* dq, float* dkk, float* dvv, float* dla,
+                            float* dbeta, float* d_init, void* workspace, cudaStream_t stream);
 size_t backward_workspace_bytes(int n_seq, long long tokens, int H, int dk, int dv);
 
 static bool head_size_ok(int d) { return d == 64 || d == 128; }
@@ -188,16 +188,16 @@ size_t kda_backward_workspace_bytes(int n_seq, int64_t tokens, int H, int dk, in
   return kda::backward_workspace_bytes(n_seq, (long long)tokens, H, dk, dv);
 }
 
-kda_status kda_backward(const void* q, const void* k, const void* v, const float* log_alpha,
-                        const float* beta, const float* init_state, const int32_t* cu_seqlens,
-                        int n_seq, int B, int T, int H, int dk, int dv, kda_dtype dtype,
-                        kda_gate gate, const void* d_o, const float* d_final, float* dq,
-                        float* dk_out, float* dv_out, float* dlog_alpha, float* dbeta,
-                        float* d_init, void* workspace, size_t workspace_bytes,
-                        cudaStream_t stream) {
+kda_status kda_backward_ex(const void* q, const void* k, const void* v, const float* log_alpha,
+                           const float* beta, const float* init_state,
+                           const int32_t* cu_seqlens, int n_seq, int B, int T, int H, int dk,
+                           int dv, kda_dtype dtype, kda_gate gate, unsigned flags,
+                           const void* d_o, const float* d_final, float* dq, float* dk_out,
+                           float* dv_out, float* dlog_alpha, float* dbeta, float* d_init,
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (B < 0 || T < 0 || H <= 0 || n_seq < 0) return KDA_ERR_INVALID_ARG;
   if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_INVALID_ARG;
-  if (!kda::gate_ok(gate)) return KDA_ERR_INVALID_ARG;
+  if (!kda::gate_ok(gate) || (flags & ~kda::kAllFlags)) return KDA_ERR_INVALID_ARG;
   if (!kda::head_size_ok(dk) || !kda::head_size_ok(dv)) return KDA_ERR_UNSUPPORTED;
   if (cu_seqlens) {
     if (B != 1) return KDA_ERR_INVALID_ARG;
@@ -222,9 +222,21 @@ kda_status kda_backward(const void* q, const void* k, const void* v, const float
   if (reinterpret_cast<uintptr_t>(workspace) & 255) return KDA_ERR_WORKSPACE;
   const cudaError_t err = kda::launch_backward(
       q, k, v, log_alpha, beta, init_state, cu_seqlens, d_o, d_final, n_seq, T, H, dk, dv,
-      dtype == KDA_BF16, (int)gate, tokens, dq, dk_out, dv_out, dlog_alpha, dbeta, d_init,
-      workspace, stream);
+      dtype == KDA_BF16, (int)gate, flags, tokens, dq, dk_out, dv_out, dlog_alpha, dbeta,
+      d_init, workspace, stream);
   return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_backward(const void* q, const void* k, const void* v, const float* log_alpha,
+                        const float* beta, const float* init_state, const int32_t* cu_seqlens,
+                        int n_seq, int B, int T, int H, int dk, int dv, kda_dtype dtype,
+                        kda_gate gate, const void* d_o, const float* d_final, float* dq,
+                        float* dk_out, float* dv_out, float* dlog_alpha, float* dbeta,
+                        float* d_init, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream) {
+  return kda_backward_ex(q, k, v, log_alpha, beta, init_state, cu_seqlens, n_seq, B, T, H, dk,
+                         dv, dtype, gate, 0u, d_o, d_final, dq, dk_out, dv_out, dlog_alpha,
+                         dbeta, d_init, workspace, workspace_bytes, stream);
 }
 
 kda_status kda_get_device_status(int reset, int* detail, cudaStream_t stream) {

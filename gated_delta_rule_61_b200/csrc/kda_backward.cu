@@ -36,12 +36,24 @@
 // one is processed). S' is recovered as S_t - k d^T with d kept from the
 // recomputation. Each block's inputs are staged in shared memory once, so
 // the per-token steps wait on no global load.
+//
+// Input prologue (raw projections, as in the forward's flags): the staging
+// applies it (q and k through SiLU and the per-token L2 normalisation, beta
+// and the decay through the sigmoid), the token steps then give the
+// gradients with respect to the transformed inputs, and a small second
+// kernel carries them back to the raw ones: through the normalisation's
+// Jacobian (I - n n^T) / max(|u|, 1e-12) and SiLU's derivative
+// s (1 + x (1 - s)) for q and k, sigmoid's s (1 - s) for beta, and
+// d log sigmoid(x) / dx = sigmoid(-x) for the gate.
 #include "kda_common.cuh"
 
 namespace kda {
 namespace bwd {
 
 constexpr int kBlk = 16;       // tokens per checkpoint block
+constexpr unsigned kRawQK = 1u, kRawBeta = 2u, kRawGate = 4u;   // prologue flags
+
+__device__ __forceinline__ float sigm(float x) { return 1.0f / (1.0f + expf(-x)); }
 constexpr int kColsWide = 32, kColsNarrow = 8;   // value columns per CTA
 
 // Sum over the warp of 32 per-lane vectors of N values (N a power of two,
@@ -71,13 +83,15 @@ __device__ __forceinline__ void red_add(float* p, float x) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(x) : "memory");
 }
 
-template <typename TIn, int DK, int DV, int kCols>
+// kPro: the inputs are raw projections (flags); without it the kernel is
+// the plain reverse sweep on ready inputs.
+template <typename TIn, int DK, int DV, int kCols, bool kPro>
 __global__ void __launch_bounds__(DK, kCols == kColsNarrow ? 1024 / DK : 2)
 backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
                 const float* __restrict__ log_alpha, const float* __restrict__ beta,
                 const float* __restrict__ init_state, const int32_t* __restrict__ cu_seqlens,
                 const TIn* __restrict__ d_o, const float* __restrict__ d_final, int T, int H,
-                int gate, float* __restrict__ dq, float* __restrict__ dk,
+                int gate, unsigned flags, float* __restrict__ dq, float* __restrict__ dk,
                 float* __restrict__ dv, float* __restrict__ dla, float* __restrict__ dbeta,
                 float* __restrict__ d_init, float* __restrict__ ckpt, float* __restrict__ scratch) {
   constexpr int kSlices = DV / kCols;
@@ -107,15 +121,32 @@ backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
   __shared__ float s_beta[kBlk];
   __shared__ float s_part[kWarps][kCols];
   __shared__ float s_d[kBlk][kCols], s_vr[kBlk][kCols];   // d_j and v_j - r_j per token
+  __shared__ float s_ik[kBlk], s_iq[kBlk];   // raw q, k: 1 / max(|SiLU(x)|, 1e-12) per token
+  const bool raw_qk = kPro && (flags & kRawQK);
 
   auto stage = [&](long long tb, int nb, bool with_q) {
     __syncthreads();   // the previous block's values are no longer read
     for (int s = 0; s < nb; ++s) {
       const size_t tok = (size_t)(tb + s) * H + head;
-      s_k[s][i] = Io<TIn>::load(k + tok * DK + i);
-      if (with_q) s_q[s][i] = Io<TIn>::load(q + tok * DK + i);
-      s_a[s][i] = gate == 0 ? expf(__ldg(log_alpha + tok * DK + i))
-                : gate == 1 ? expf(__ldg(log_alpha + tok)) : 1.f;
+      if constexpr (kPro) {
+        const float kx = Io<TIn>::load(k + tok * DK + i);
+        s_k[s][i] = raw_qk ? kx * sigm(kx) : kx;
+        if (with_q) {
+          const float qx = Io<TIn>::load(q + tok * DK + i);
+          s_q[s][i] = raw_qk ? qx * sigm(qx) : qx;
+        }
+        float a = 1.f;
+        if (gate != 2) {
+          const float x = gate == 0 ? __ldg(log_alpha + tok * DK + i) : __ldg(log_alpha + tok);
+          a = (flags & kRawGate) ? sigm(x) : expf(x);   // exp(log sigmoid(x)) = sigmoid(x)
+        }
+        s_a[s][i] = a;
+      } else {
+        s_k[s][i] = Io<TIn>::load(k + tok * DK + i);
+        if (with_q) s_q[s][i] = Io<TIn>::load(q + tok * DK + i);
+        s_a[s][i] = gate == 0 ? expf(__ldg(log_alpha + tok * DK + i))
+                  : gate == 1 ? expf(__ldg(log_alpha + tok)) : 1.f;
+      }
     }
     for (int e = i; e < nb * kCols; e += DK) {
       const int s = e / kCols, j = e - (e / kCols) * kCols;
@@ -123,8 +154,37 @@ backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
       s_v[s][j] = Io<TIn>::load(v + tok * DV + col0 + j);
       if (with_q) s_do[s][j] = Io<TIn>::load(d_o + tok * DV + col0 + j);
     }
-    if (i < nb) s_beta[i] = __ldg(beta + (size_t)(tb + i) * H + head);
+    if (i < nb) {
+      const float b = __ldg(beta + (size_t)(tb + i) * H + head);
+      s_beta[i] = (kPro && (flags & kRawBeta)) ? sigm(b) : b;
+    }
     __syncthreads();
+    if (kPro && raw_qk) {
+      // per-token L2 norms of SiLU(k), SiLU(q) over the key rows: warp w
+      // takes tokens w, w + kWarps, ...
+      for (int s = warp; s < nb; s += kWarps) {
+        float nk = 0.f, nq = 0.f;
+        for (int r = lane; r < DK; r += 32) {
+          nk = fmaf(s_k[s][r], s_k[s][r], nk);
+          if (with_q) nq = fmaf(s_q[s][r], s_q[s][r], nq);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          nk += __shfl_xor_sync(0xffffffffu, nk, off);
+          nq += __shfl_xor_sync(0xffffffffu, nq, off);
+        }
+        if (lane == 0) {
+          s_ik[s] = 1.f / fmaxf(sqrtf(nk), 1e-12f);
+          s_iq[s] = 1.f / fmaxf(sqrtf(nq), 1e-12f);
+        }
+      }
+      __syncthreads();
+      for (int s = 0; s < nb; ++s) {
+        s_k[s][i] *= s_ik[s];
+        if (with_q) s_q[s][i] *= s_iq[s];
+      }
+      __syncthreads();
+    }
   };
 
   const size_t state_off = ((size_t)seq * H + head) * DK * DV + (size_t)i * DV + col0;
@@ -282,6 +342,71 @@ backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
   }
 }
 
+// The prologue's reverse mode, after the token steps: one warp per (token,
+// head) row. The gradients with respect to the transformed inputs (in dq, dk,
+// dbeta, dlog_alpha) become those with respect to the raw inputs, in place.
+template <typename TIn, int DK>
+__global__ void __launch_bounds__(256)
+prologue_vjp_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
+                    const float* __restrict__ log_alpha, const float* __restrict__ beta,
+                    long long rows, int gate, unsigned flags, float* __restrict__ dq,
+                    float* __restrict__ dk, float* __restrict__ dla,
+                    float* __restrict__ dbeta) {
+  constexpr int NJ = DK / 32;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);   // token * H + head
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;   // the whole warp leaves together
+  if (flags & kRawQK) {
+#pragma unroll 1
+    for (int which = 0; which < 2; ++which) {
+      const TIn* x = which ? k : q;
+      float* g = which ? dk : dq;
+      float xv[NJ], sv[NJ], uv[NJ], gv[NJ], uu = 0.f;
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const size_t idx = (size_t)row * DK + lane + 32 * j;
+        xv[j] = Io<TIn>::load(x + idx);
+        sv[j] = sigm(xv[j]);
+        uv[j] = xv[j] * sv[j];
+        gv[j] = g[idx];
+        uu = fmaf(uv[j], uv[j], uu);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) uu += __shfl_xor_sync(0xffffffffu, uu, off);
+      uu = __shfl_sync(0xffffffffu, uu, 0);
+      const float r = sqrtf(uu), inv = 1.f / fmaxf(r, 1e-12f);
+      // n . g with n = u / max(|u|, 1e-12)
+      float dot = 0.f;
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) dot = fmaf(uv[j] * inv, gv[j], dot);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+      dot = __shfl_sync(0xffffffffu, dot, 0);
+      const bool proj = r > 1e-12f;   // below it the map is u / 1e-12, a plain scale
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const float du = (proj ? fmaf(-uv[j] * inv, dot, gv[j]) : gv[j]) * inv;
+        g[(size_t)row * DK + lane + 32 * j] = du * sv[j] * fmaf(xv[j], 1.f - sv[j], 1.f);
+      }
+    }
+  }
+  if ((flags & kRawBeta) && lane == 0) {
+    const float sb = sigm(__ldg(beta + row));
+    dbeta[row] *= sb * (1.f - sb);
+  }
+  if (flags & kRawGate) {
+    if (gate == 0) {
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const size_t idx = (size_t)row * DK + lane + 32 * j;
+        dla[idx] *= sigm(-__ldg(log_alpha + idx));
+      }
+    } else if (gate == 1 && lane == 0) {
+      dla[row] *= sigm(-__ldg(log_alpha + row));
+    }
+  }
+}
+
 }  // namespace bwd
 
 // Workspace: checkpoints (floor(tokens / 16) + n_seq + 1 blocks per head, each
@@ -299,23 +424,30 @@ template <typename TIn, int DK, int DV>
 static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, const float* la,
                                 const float* beta, const float* s0, const int32_t* cu,
                                 const void* d_o, const float* d_final, int n_seq, int T, int H,
-                                int gate, float* dq, float* dk, float* dv, float* dla,
-                                float* dbeta, float* d_init, float* ckpt, float* scratch,
-                                cudaStream_t stream) {
+                                int gate, unsigned flags, long long tokens, float* dq, float* dk,
+                                float* dv, float* dla, float* dbeta, float* d_init, float* ckpt,
+                                float* scratch, cudaStream_t stream) {
   // Few chains: narrow slices, so that enough CTAs run to hide the per-token
   // latency of each chain (2 x 148 CTAs of the wide slices fill a B200).
   const long long chains = (long long)n_seq * H;
-  if (chains * (DV / bwd::kColsWide) < 2 * 148) {
-    constexpr int kC = bwd::kColsNarrow;
-    bwd::backward_kernel<TIn, DK, DV, kC><<<(unsigned)(chains * (DV / kC)), DK, 0, stream>>>(
-        (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, s0, cu, (const TIn*)d_o, d_final,
-        T, H, gate, dq, dk, dv, dla, dbeta, d_init, ckpt, scratch);
+  const bool narrow = chains * (DV / bwd::kColsWide) < 2 * 148;
+#define KDA_BWD_LAUNCH(kC, kPro)                                                               \
+  bwd::backward_kernel<TIn, DK, DV, kC, kPro><<<(unsigned)(chains * (DV / kC)), DK, 0, stream>>>( \
+      (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, s0, cu, (const TIn*)d_o, d_final,   \
+      T, H, gate, flags, dq, dk, dv, dla, dbeta, d_init, ckpt, scratch)
+  if (narrow) {
+    if (flags) KDA_BWD_LAUNCH(bwd::kColsNarrow, true);
+    else KDA_BWD_LAUNCH(bwd::kColsNarrow, false);
   } else {
-    constexpr int kC = bwd::kColsWide;
-    bwd::backward_kernel<TIn, DK, DV, kC><<<(unsigned)(chains * (DV / kC)), DK, 0, stream>>>(
-        (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, s0, cu, (const TIn*)d_o, d_final,
-        T, H, gate, dq, dk, dv, dla, dbeta, d_init, ckpt, scratch);
+    if (flags) KDA_BWD_LAUNCH(bwd::kColsWide, true);
+    else KDA_BWD_LAUNCH(bwd::kColsWide, false);
   }
+#undef KDA_BWD_LAUNCH
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || flags == 0u || tokens == 0) return e;
+  const long long rows = tokens * H;
+  bwd::prologue_vjp_kernel<TIn, DK><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+      (const TIn*)q, (const TIn*)k, la, beta, rows, gate, flags, dq, dk, dla, dbeta);
   return cudaGetLastError();
 }
 
@@ -323,7 +455,8 @@ static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, con
 cudaError_t launch_backward(const void* q, const void* k, const void* v, const float* la,
                             const float* beta, const float* s0, const int32_t* cu,
                             const void* d_o, const float* d_final, int n_seq, int T, int H,
-                            int dk, int dv, bool bf16, int gate, long long tokens, float* dq,
+                            int dk, int dv, bool bf16, int gate, unsigned flags, long long tokens,
+                            float* dq,
                             float* dkk, float* dvv, float* dla, float* dbeta, float* d_init,
                             void* workspace, cudaStream_t stream) {
   if (n_seq == 0) return cudaSuccess;
@@ -341,8 +474,8 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const f
   const size_t ck = blocks * (size_t)H * dk * dv * sizeof(float);
   float* ckpt = static_cast<float*>(workspace);
   float* scratch = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + (ck + 255) / 256 * 256);
-#define KDA_BWD_ARGS q, k, v, la, beta, s0, cu, d_o, d_final, n_seq, T, H, gate, dq, dkk, dvv, dla, \
-                     dbeta, d_init, ckpt, scratch, stream
+#define KDA_BWD_ARGS q, k, v, la, beta, s0, cu, d_o, d_final, n_seq, T, H, gate, flags, tokens, dq, \
+                     dkk, dvv, dla, dbeta, d_init, ckpt, scratch, stream
   if (bf16) {
     if (dk == 128 && dv == 128) return launch_bwd_t<__nv_bfloat16, 128, 128>(KDA_BWD_ARGS);
     if (dk == 128 && dv == 64) return launch_bwd_t<__nv_bfloat16, 128, 64>(KDA_BWD_ARGS);

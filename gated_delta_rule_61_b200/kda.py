@@ -27,7 +27,8 @@ DECODE_MAX_TOKENS = 16
 
 EXPORTS = ("kda_status_string", "kda_version", "kda_prefill_workspace_bytes",
            "kda_prefill", "kda_prefill_ex", "kda_decode_step", "kda_decode_ex",
-           "kda_backward_workspace_bytes", "kda_backward", "kda_prefill_noalloc",
+           "kda_backward_workspace_bytes", "kda_backward", "kda_backward_ex",
+           "kda_prefill_noalloc",
            "kda_get_device_status", "kda_selftest_wait_timeout")
 NOALLOC_MAX_SEQS = 65536
 
@@ -75,6 +76,10 @@ def lib():
                                ctypes.c_int, ctypes.c_int, vp, fp, fp, fp, fp, fp, fp, fp,
                                vp, ctypes.c_size_t, vp]
     L.kda_backward.restype = ctypes.c_int
+    L.kda_backward_ex.argtypes = [vp, vp, vp, fp, fp, fp, i32p, ip, ip, ip, ip, ip, ip,
+                                  ctypes.c_int, ctypes.c_int, ctypes.c_uint, vp, fp, fp, fp, fp,
+                                  fp, fp, fp, vp, ctypes.c_size_t, vp]
+    L.kda_backward_ex.restype = ctypes.c_int
     L.kda_prefill_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, i32p, ip, ip, ip, vp, fp, vp]
     L.kda_prefill_noalloc.restype = ctypes.c_int
     L.kda_get_device_status.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int), vp]
@@ -196,11 +201,14 @@ def prefill(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, *, chunk
 
 
 def backward(q, k, v, log_alpha, beta, d_o, init_state=None, cu_seqlens=None, d_final=None,
-             *, gate="channel", workspace=None, stream=None):
-    """Gradients through the recurrence (kda_backward): returns a dict of fp32
-    tensors dq, dk, dv, dlog_alpha (None for gate "none"), dbeta and d_init
-    ([N, H, dk, dv]). Inputs as for prefill (ready inputs, no prologue);
-    d_o shaped like v in v's dtype; d_final [N, H, dk, dv] fp32 or None."""
+             *, gate="channel", raw_qk=False, raw_beta=False, raw_gate=False, workspace=None,
+             stream=None):
+    """Gradients through the recurrence (kda_backward_ex): returns a dict of
+    fp32 tensors dq, dk, dv, dlog_alpha (None for gate "none"), dbeta and
+    d_init ([N, H, dk, dv]). Inputs as for prefill, including the prologue
+    flags (the gradients are then with respect to the raw projections and
+    logits); d_o shaped like v in v's dtype; d_final [N, H, dk, dv] fp32 or
+    None."""
     if gate not in GATES:
         raise ValueError("gate must be one of %s" % list(GATES))
     B, T, H, dk = q.shape
@@ -235,14 +243,15 @@ def backward(q, k, v, log_alpha, beta, d_o, init_state=None, cu_seqlens=None, d_
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
     ws_bytes = workspace.numel() * workspace.element_size()
-    st = lib().kda_backward(
+    st = lib().kda_backward_ex(
         _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(init_state),
         _ptr(cu_seqlens), int(n_seq), int(B), int(T), int(H), int(dk), int(dv), code,
-        GATES[gate], _ptr(d_o), _ptr(d_final), _ptr(out["dq"]), _ptr(out["dk"]),
+        GATES[gate], _flags(raw_qk, raw_beta, raw_gate), _ptr(d_o), _ptr(d_final),
+        _ptr(out["dq"]), _ptr(out["dk"]),
         _ptr(out["dv"]), _ptr(out["dlog_alpha"]), _ptr(out["dbeta"]), _ptr(out["d_init"]),
         _ptr(workspace), ws_bytes, _stream(stream))
     if st != KDA_OK:
-        raise KdaError(st, "kda_backward")
+        raise KdaError(st, "kda_backward_ex")
     return out
 
 

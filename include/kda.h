@@ -233,7 +233,8 @@ kda_status kda_decode_ex(const void *q, const void *k, const void *v,
  * The gate is applied exactly (no clamp). Work: a forward pass that stores
  * the state every 16 tokens in the workspace, then a reverse sweep that
  * recomputes each 16-token block from its checkpoint (token-recurrent, one
- * CTA per (sequence, head, 32 value columns)). The column slices of a head
+ * CTA per (sequence, head, slice of value columns: 32 wide, or 8 when the
+ * sequences and heads are few)). The column slices of a head
  * add their parts of dq, dk, dlog_alpha and dbeta with atomic adds, so those
  * can differ between runs in the last bits. init_state, d_final and d_init
  * must be 16-byte aligned. workspace: at least
@@ -251,6 +252,32 @@ kda_status kda_backward(const void *q, const void *k, const void *v,
                         float *dq, float *dk_out, float *dv_out, float *dlog_alpha,
                         float *dbeta, float *d_init,
                         void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * kda_backward_ex -- kda_backward for inputs given as raw projections: the
+ * reverse mode of kda_prefill_ex with the same prologue flags (KDA_RAW_QK,
+ * KDA_RAW_BETA, KDA_RAW_GATE; the cached forward of "DeltaNet, or Fast Weight
+ * Programmers" applies SiLU and L2 normalisation to q and k and a sigmoid to
+ * beta before the recurrence). The gradients returned are with respect to the
+ * inputs as passed: dq, dk_out through the normalisation's Jacobian
+ * (I - n n^T) / max(|u|, 1e-12) (u = SiLU(x), n = u / max(|u|, 1e-12); below
+ * 1e-12 the map is u / 1e-12) and SiLU's derivative; dbeta through the
+ * sigmoid; dlog_alpha, for gate logits x, is dL/dx = dL/dlog_alpha times
+ * sigmoid(-x). The prologue runs in fp32 inside the kernels (exact expf-based
+ * SiLU and sigmoid); a second kernel on the same stream maps the gradients
+ * back to the raw inputs after the token sweep. flags 0 is kda_backward.
+ * Arguments, layouts, workspace and errors otherwise as kda_backward; flags
+ * other than the three: KDA_ERR_INVALID_ARG.
+ */
+kda_status kda_backward_ex(const void *q, const void *k, const void *v,
+                           const float *log_alpha, const float *beta,
+                           const float *init_state, const int32_t *cu_seqlens,
+                           int n_seq, int B, int T, int H, int dk, int dv,
+                           kda_dtype dtype, kda_gate gate, unsigned flags,
+                           const void *d_o, const float *d_final,
+                           float *dq, float *dk_out, float *dv_out, float *dlog_alpha,
+                           float *dbeta, float *d_init,
+                           void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * kda_prefill_noalloc -- the packed variable-length chunked prefill of

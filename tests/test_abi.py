@@ -124,6 +124,27 @@ def test_decode_rejects_bad_arguments(kw, status):
     assert _decode(**kw) == status
 
 
+def _backward(**kw):
+    a = dict(B=2, T=4, H=2, dk=128, dv=128, dtype=kda.KDA_BF16, gate=kda.KDA_GATE_CHANNEL,
+             flags=0, ws=None, ws_bytes=0)
+    a.update(kw)
+    return kda.lib().kda_backward_ex(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 0, a["B"], a["T"],
+                                     a["H"], a["dk"], a["dv"], a["dtype"], a["gate"], a["flags"],
+                                     FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, None, a["ws"],
+                                     a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(flags=8), kda.KDA_ERR_INVALID_ARG),         # not a prologue flag
+    (dict(gate=7), kda.KDA_ERR_INVALID_ARG),
+    (dict(dk=100), kda.KDA_ERR_UNSUPPORTED),
+    (dict(flags=7), kda.KDA_ERR_WORKSPACE),           # valid flags; no workspace given
+    (dict(B=0, T=0), kda.KDA_OK),
+])
+def test_backward_rejects_bad_arguments(kw, status):
+    assert _backward(**kw) == status
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device error path")
 def test_launch_without_device_reports_cuda_error():
     assert _decode() == kda.KDA_ERR_CUDA

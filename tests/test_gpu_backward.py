@@ -99,3 +99,53 @@ def test_backward_long_sequence_many_blocks():
 def test_backward_many_chains_wide_slices():
     # enough chains that each CTA takes 32 value columns (few chains take 8)
     _check(_case(2, 40, 80, 128, 128, torch.float32, "channel", seed=13), "channel")
+
+
+def _raw_case(B, T, H, d, dtype, gate, seed, lengths=None):
+    """The same case with raw projections: q, k ~ N(0, 1) unnormalised, beta
+    logits ~ N(0, 1), gate logits ~ N(3, 1) (decays sigmoid(x) near 0.95)."""
+    inp = _case(B, T, H, d, d, dtype, gate, seed, lengths=lengths)
+    g = torch.Generator().manual_seed(seed + 1)
+    shape = inp["q"].shape
+    inp["q"] = torch.randn(shape, generator=g).to(dtype)
+    inp["k"] = torch.randn(shape, generator=g).to(dtype)
+    inp["beta"] = torch.randn(inp["beta"].shape, generator=g)
+    if inp["log_alpha"] is not None:
+        inp["log_alpha"] = torch.randn(inp["log_alpha"].shape, generator=g) + 3.0
+    return inp
+
+
+def _check_raw(inp, gate, tol=TOL_F32):
+    cu = inp["cu_seqlens"]
+    names = ("q", "k", "v", "log_alpha", "beta", "d_o")
+    if cu is not None:
+        args = [None if inp[n] is None else inp[n][0] for n in names]
+        cu = cu.numpy().astype(np.int64)
+    else:
+        args = [inp[n] for n in names]
+    ref = oracle.kda_backward_ex(*args, init_state=inp["init_state"], d_final=inp["d_final"],
+                                 cu_seqlens=cu, gate=gate, raw_qk=True, raw_beta=True,
+                                 raw_gate=True)
+    c = {n: (x.cuda() if isinstance(x, torch.Tensor) else x) for n, x in inp.items()}
+    out = kda.backward(c["q"], c["k"], c["v"], c["log_alpha"], c["beta"], c["d_o"],
+                       init_state=c["init_state"], cu_seqlens=c["cu_seqlens"],
+                       d_final=c["d_final"], gate=gate, raw_qk=True, raw_beta=True,
+                       raw_gate=True)
+    torch.cuda.synchronize()
+    for n in ("dq", "dk", "dv", "dbeta", "d_init") + (("dlog_alpha",) if gate != "none" else ()):
+        r = ref[n][None] if cu is not None and n != "d_init" else ref[n]
+        assert_close(out[n], r, tol, "backward through the prologue %s (gate %s)" % (n, gate))
+
+
+@pytest.mark.parametrize("gate", ["channel", "scalar", "none"])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_backward_through_the_prologue(gate, dtype):
+    """Raw projections (SiLU + L2 normalisation of q and k, beta and gate
+    logits): kda_backward_ex against the oracle's reverse mode through the
+    same prologue."""
+    _check_raw(_raw_case(2, 45, 3, 128, dtype, gate, seed=21 + len(gate)), gate)
+
+
+def test_backward_through_the_prologue_packed_and_small_heads():
+    _check_raw(_raw_case(1, 0, 2, 64, torch.float32, "channel", seed=23,
+                         lengths=[5, 0, 33, 17]), "channel")
