@@ -166,3 +166,41 @@ def test_backward_ex_without_prologue_is_the_plain_reverse_mode():
     for n in ("dq", "dk", "dv", "dbeta", "d_init"):
         np.testing.assert_array_equal(g[n], ref[n])
     np.testing.assert_array_equal(g["dlog_alpha"], ref["dlog_alpha"].sum(-1))
+
+
+def test_prologue_pin_catches_a_planted_mistake(monkeypatch):
+    """The finite-difference pin above is sharp: the normalisation's Jacobian
+    without its projection term (a plausible slip) moves dq and dk far
+    outside its tolerance."""
+    def wrong_vjp(x, g, eps=1e-12):
+        x, g = oracle._f64(x), oracle._f64(g)
+        s = oracle.sigmoid(x)
+        u = x * s
+        r = np.sqrt(np.sum(u * u, axis=-1, keepdims=True))
+        return g / np.maximum(r, eps) * s * (1.0 + x * (1.0 - s))
+
+    rng = np.random.default_rng(41)
+    T, H, dk, dv = 4, 1, 5, 3
+    q, k = rng.standard_normal((T, H, dk)), rng.standard_normal((T, H, dk))
+    v = rng.standard_normal((T, H, dv))
+    b = rng.standard_normal((T, H))
+    Wo = rng.standard_normal((T, H, dv))
+
+    def loss(qq):
+        o, _ = oracle.kda_forward_ex(qq, k, v, None, b, gate="none", raw_qk=True, raw_beta=True)
+        return float(np.sum(o * Wo))
+
+    h = 1e-6
+    num = np.zeros_like(q)
+    for idx in np.ndindex(*q.shape):
+        qp, qm = q.copy(), q.copy()
+        qp[idx] += h
+        qm[idx] -= h
+        num[idx] = (loss(qp) - loss(qm)) / (2 * h)
+    good = oracle.kda_backward_ex(q, k, v, None, b, Wo, gate="none", raw_qk=True,
+                                  raw_beta=True)["dq"]
+    np.testing.assert_allclose(good, num, rtol=1e-6, atol=1e-7)
+    monkeypatch.setattr(oracle, "_prologue_qk_vjp", wrong_vjp)
+    bad = oracle.kda_backward_ex(q, k, v, None, b, Wo, gate="none", raw_qk=True,
+                                 raw_beta=True)["dq"]
+    assert np.max(np.abs(bad - num)) > 1e-3
