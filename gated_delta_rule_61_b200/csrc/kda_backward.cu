@@ -37,11 +37,13 @@
 // recomputation. Each block's inputs are staged in shared memory once, so
 // the per-token steps wait on no global load.
 //
-// Input prologue (raw projections, as in the forward's flags): the staging
-// applies it (q and k through SiLU and the per-token L2 normalisation, beta
-// and the decay through the sigmoid), the token steps then give the
-// gradients with respect to the transformed inputs, and a small second
-// kernel carries them back to the raw ones: through the normalisation's
+// Input prologue (raw projections, as in the forward's flags): a small first
+// kernel stores each (token, head) row's 1 / max(|SiLU(q)|, 1e-12) and the
+// same for k in the workspace; the staging applies the prologue with them
+// (q and k through SiLU and that scale, beta and the decay through the
+// sigmoid), the token steps then give the gradients with respect to the
+// transformed inputs, and a last kernel carries them back to the raw ones:
+// through the normalisation's
 // Jacobian (I - n n^T) / max(|u|, 1e-12) and SiLU's derivative
 // s (1 + x (1 - s)) for q and k, sigmoid's s (1 - s) for beta, and
 // d log sigmoid(x) / dx = sigmoid(-x) for the gate.
@@ -54,6 +56,9 @@ constexpr int kBlk = 16;       // tokens per checkpoint block
 constexpr unsigned kRawQK = 1u, kRawBeta = 2u, kRawGate = 4u;   // prologue flags
 
 __device__ __forceinline__ float sigm(float x) { return 1.0f / (1.0f + expf(-x)); }
+// the staging's sigmoid: approximate exponential and reciprocal (relative
+// error a few 1e-7, far below the gradients' tolerance; 1 / inf = 0)
+__device__ __forceinline__ float sigm_fast(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
 constexpr int kColsWide = 32, kColsNarrow = 8;   // value columns per CTA
 
 // Sum over the warp of 32 per-lane vectors of N values (N a power of two,
@@ -91,7 +96,8 @@ backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
                 const float* __restrict__ log_alpha, const float* __restrict__ beta,
                 const float* __restrict__ init_state, const int32_t* __restrict__ cu_seqlens,
                 const TIn* __restrict__ d_o, const float* __restrict__ d_final, int T, int H,
-                int gate, unsigned flags, float* __restrict__ dq, float* __restrict__ dk,
+                int gate, unsigned flags, const float* __restrict__ inv_norm,
+                float* __restrict__ dq, float* __restrict__ dk,
                 float* __restrict__ dv, float* __restrict__ dla, float* __restrict__ dbeta,
                 float* __restrict__ d_init, float* __restrict__ ckpt, float* __restrict__ scratch) {
   constexpr int kSlices = DV / kCols;
@@ -121,7 +127,6 @@ backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
   __shared__ float s_beta[kBlk];
   __shared__ float s_part[kWarps][kCols];
   __shared__ float s_d[kBlk][kCols], s_vr[kBlk][kCols];   // d_j and v_j - r_j per token
-  __shared__ float s_ik[kBlk], s_iq[kBlk];   // raw q, k: 1 / max(|SiLU(x)|, 1e-12) per token
   const bool raw_qk = kPro && (flags & kRawQK);
 
   auto stage = [&](long long tb, int nb, bool with_q) {
@@ -129,16 +134,18 @@ backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
     for (int s = 0; s < nb; ++s) {
       const size_t tok = (size_t)(tb + s) * H + head;
       if constexpr (kPro) {
+        // raw q, k: SiLU(x) / max(|SiLU(x)|, 1e-12), the row's scale from the
+        // first kernel (inv_norm[2 row] for q, [2 row + 1] for k)
         const float kx = Io<TIn>::load(k + tok * DK + i);
-        s_k[s][i] = raw_qk ? kx * sigm(kx) : kx;
+        s_k[s][i] = raw_qk ? kx * sigm_fast(kx) * __ldg(inv_norm + 2 * tok + 1) : kx;
         if (with_q) {
           const float qx = Io<TIn>::load(q + tok * DK + i);
-          s_q[s][i] = raw_qk ? qx * sigm(qx) : qx;
+          s_q[s][i] = raw_qk ? qx * sigm_fast(qx) * __ldg(inv_norm + 2 * tok) : qx;
         }
         float a = 1.f;
         if (gate != 2) {
           const float x = gate == 0 ? __ldg(log_alpha + tok * DK + i) : __ldg(log_alpha + tok);
-          a = (flags & kRawGate) ? sigm(x) : expf(x);   // exp(log sigmoid(x)) = sigmoid(x)
+          a = (flags & kRawGate) ? sigm_fast(x) : expf(x);   // exp(log sigmoid(x)) = sigmoid(x)
         }
         s_a[s][i] = a;
       } else {
@@ -156,35 +163,9 @@ backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
     }
     if (i < nb) {
       const float b = __ldg(beta + (size_t)(tb + i) * H + head);
-      s_beta[i] = (kPro && (flags & kRawBeta)) ? sigm(b) : b;
+      s_beta[i] = (kPro && (flags & kRawBeta)) ? sigm_fast(b) : b;
     }
     __syncthreads();
-    if (kPro && raw_qk) {
-      // per-token L2 norms of SiLU(k), SiLU(q) over the key rows: warp w
-      // takes tokens w, w + kWarps, ...
-      for (int s = warp; s < nb; s += kWarps) {
-        float nk = 0.f, nq = 0.f;
-        for (int r = lane; r < DK; r += 32) {
-          nk = fmaf(s_k[s][r], s_k[s][r], nk);
-          if (with_q) nq = fmaf(s_q[s][r], s_q[s][r], nq);
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          nk += __shfl_xor_sync(0xffffffffu, nk, off);
-          nq += __shfl_xor_sync(0xffffffffu, nq, off);
-        }
-        if (lane == 0) {
-          s_ik[s] = 1.f / fmaxf(sqrtf(nk), 1e-12f);
-          s_iq[s] = 1.f / fmaxf(sqrtf(nq), 1e-12f);
-        }
-      }
-      __syncthreads();
-      for (int s = 0; s < nb; ++s) {
-        s_k[s][i] *= s_ik[s];
-        if (with_q) s_q[s][i] *= s_iq[s];
-      }
-      __syncthreads();
-    }
   };
 
   const size_t state_off = ((size_t)seq * H + head) * DK * DV + (size_t)i * DV + col0;
@@ -342,6 +323,35 @@ backward_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn*
   }
 }
 
+// 1 / max(|SiLU(x)|, 1e-12) of every (token, head) row of raw q and k (one
+// warp per row), into inv_norm[2 row] (q) and inv_norm[2 row + 1] (k).
+template <typename TIn, int DK>
+__global__ void __launch_bounds__(256)
+prologue_norms_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k, long long rows,
+                      float* __restrict__ inv_norm) {
+  constexpr int NJ = DK / 32;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;   // the whole warp leaves together
+  float nq = 0.f, nk = 0.f;
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    const size_t idx = (size_t)row * DK + lane + 32 * j;
+    const float xq = Io<TIn>::load(q + idx), xk = Io<TIn>::load(k + idx);
+    const float uq = xq * sigm(xq), uk = xk * sigm(xk);
+    nq = fmaf(uq, uq, nq);
+    nk = fmaf(uk, uk, nk);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    nq += __shfl_xor_sync(0xffffffffu, nq, off);
+    nk += __shfl_xor_sync(0xffffffffu, nk, off);
+  }
+  if (lane == 0)
+    *reinterpret_cast<float2*>(inv_norm + 2 * row) =
+        make_float2(1.f / fmaxf(sqrtf(nq), 1e-12f), 1.f / fmaxf(sqrtf(nk), 1e-12f));
+}
+
 // The prologue's reverse mode, after the token steps: one warp per (token,
 // head) row. The gradients with respect to the transformed inputs (in dq, dk,
 // dbeta, dlog_alpha) become those with respect to the raw inputs, in place.
@@ -410,14 +420,18 @@ prologue_vjp_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
 }  // namespace bwd
 
 // Workspace: checkpoints (floor(tokens / 16) + n_seq + 1 blocks per head, each
-// dk x dv fp32) and one 16 x dk x kCols fp32 scratch per CTA (16 x dk x dv
-// per head whatever the slice width), 256-byte aligned.
+// dk x dv fp32), one 16 x dk x kCols fp32 scratch per CTA (16 x dk x dv per
+// head whatever the slice width) and, for raw q and k, two fp32 scales per
+// (token, head) row; each region 256-byte aligned.
+static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
 size_t backward_workspace_bytes(int n_seq, long long tokens, int H, int dk, int dv) {
   if (n_seq <= 0 || H <= 0) return 0;
   const size_t blocks = (size_t)(tokens / bwd::kBlk) + (size_t)n_seq + 1;
   const size_t ck = blocks * (size_t)H * dk * dv * sizeof(float);
   const size_t scr = (size_t)n_seq * H * bwd::kBlk * dk * dv * sizeof(float);
-  return (ck + 255) / 256 * 256 + (scr + 255) / 256 * 256;
+  const size_t nrm = (size_t)tokens * H * 2 * sizeof(float);
+  return align256(ck) + align256(scr) + align256(nrm);
 }
 
 template <typename TIn, int DK, int DV>
@@ -426,7 +440,14 @@ static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, con
                                 const void* d_o, const float* d_final, int n_seq, int T, int H,
                                 int gate, unsigned flags, long long tokens, float* dq, float* dk,
                                 float* dv, float* dla, float* dbeta, float* d_init, float* ckpt,
-                                float* scratch, cudaStream_t stream) {
+                                float* scratch, float* inv_norm, cudaStream_t stream) {
+  const long long rows = tokens * H;
+  if ((flags & bwd::kRawQK) && rows > 0) {
+    bwd::prologue_norms_kernel<TIn, DK><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+        (const TIn*)q, (const TIn*)k, rows, inv_norm);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   // Few chains: narrow slices, so that enough CTAs run to hide the per-token
   // latency of each chain (2 x 148 CTAs of the wide slices fill a B200).
   const long long chains = (long long)n_seq * H;
@@ -434,7 +455,7 @@ static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, con
 #define KDA_BWD_LAUNCH(kC, kPro)                                                               \
   bwd::backward_kernel<TIn, DK, DV, kC, kPro><<<(unsigned)(chains * (DV / kC)), DK, 0, stream>>>( \
       (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, s0, cu, (const TIn*)d_o, d_final,   \
-      T, H, gate, flags, dq, dk, dv, dla, dbeta, d_init, ckpt, scratch)
+      T, H, gate, flags, inv_norm, dq, dk, dv, dla, dbeta, d_init, ckpt, scratch)
   if (narrow) {
     if (flags) KDA_BWD_LAUNCH(bwd::kColsNarrow, true);
     else KDA_BWD_LAUNCH(bwd::kColsNarrow, false);
@@ -445,7 +466,6 @@ static cudaError_t launch_bwd_t(const void* q, const void* k, const void* v, con
 #undef KDA_BWD_LAUNCH
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || flags == 0u || tokens == 0) return e;
-  const long long rows = tokens * H;
   bwd::prologue_vjp_kernel<TIn, DK><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
       (const TIn*)q, (const TIn*)k, la, beta, rows, gate, flags, dq, dk, dla, dbeta);
   return cudaGetLastError();
@@ -472,10 +492,13 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const f
   }
   const size_t blocks = (size_t)(tokens / bwd::kBlk) + (size_t)n_seq + 1;
   const size_t ck = blocks * (size_t)H * dk * dv * sizeof(float);
-  float* ckpt = static_cast<float*>(workspace);
-  float* scratch = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + (ck + 255) / 256 * 256);
+  const size_t scr = (size_t)n_seq * H * bwd::kBlk * dk * dv * sizeof(float);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* ckpt = reinterpret_cast<float*>(ws);
+  float* scratch = reinterpret_cast<float*>(ws + align256(ck));
+  float* inv_norm = reinterpret_cast<float*>(ws + align256(ck) + align256(scr));
 #define KDA_BWD_ARGS q, k, v, la, beta, s0, cu, d_o, d_final, n_seq, T, H, gate, flags, tokens, dq, \
-                     dkk, dvv, dla, dbeta, d_init, ckpt, scratch, stream
+                     dkk, dvv, dla, dbeta, d_init, ckpt, scratch, inv_norm, stream
   if (bf16) {
     if (dk == 128 && dv == 128) return launch_bwd_t<__nv_bfloat16, 128, 128>(KDA_BWD_ARGS);
     if (dk == 128 && dv == 64) return launch_bwd_t<__nv_bfloat16, 128, 64>(KDA_BWD_ARGS);

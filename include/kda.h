@@ -263,9 +263,13 @@ kda_status kda_backward(const void *q, const void *k, const void *v,
  * (I - n n^T) / max(|u|, 1e-12) (u = SiLU(x), n = u / max(|u|, 1e-12); below
  * 1e-12 the map is u / 1e-12) and SiLU's derivative; dbeta through the
  * sigmoid; dlog_alpha, for gate logits x, is dL/dx = dL/dlog_alpha times
- * sigmoid(-x). The prologue runs in fp32 inside the kernels (exact expf-based
- * SiLU and sigmoid); a second kernel on the same stream maps the gradients
- * back to the raw inputs after the token sweep. flags 0 is kda_backward.
+ * sigmoid(-x). The prologue runs in fp32 inside the kernels: a first kernel
+ * stores each row's 1 / max(|SiLU(x)|, 1e-12) for q and k in the workspace,
+ * the token sweep applies SiLU and the sigmoids with the hardware exponential
+ * and reciprocal (relative error a few 1e-7), and a last kernel on the same
+ * stream maps the gradients back to the raw inputs (expf-based). flags 0 is
+ * kda_backward. The workspace (kda_backward_workspace_bytes) includes the
+ * row scales.
  * Arguments, layouts, workspace and errors otherwise as kda_backward; flags
  * other than the three: KDA_ERR_INVALID_ARG.
  */
