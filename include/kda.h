@@ -225,7 +225,7 @@ kda_status kda_decode_ex(const void *q, const void *k, const void *v,
  * forward inputs and dL/do (and optionally dL/dS_final), returns dL/dq,
  * dL/dk, dL/dv, dL/dlog_alpha, dL/dbeta and dL/dS_0, all fp32:
  *   q, k, v, log_alpha, beta, init_state, cu_seqlens, n_seq, B, T, H, dk, dv,
- *   dtype, gate   as for kda_prefill_ex (ready inputs: no prologue flags)
+ *   dtype, gate   as for kda_prefill_ex (ready inputs; raw ones: kda_backward_ex)
  *   d_o        [B, T, H, dv] dtype           d_final [n_seq, H, dk, dv] fp32 or NULL
  *   dq, dk_out [B, T, H, dk] fp32            dv_out  [B, T, H, dv] fp32
  *   dlog_alpha the gate's shape, fp32 (NULL with KDA_GATE_NONE)
