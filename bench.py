@@ -274,7 +274,7 @@ def bench_backward(args, dev, stream, hbm, world, inp):
     import torch
     from gated_delta_rule_61_b200 import kda
     P = PREFILL
-    T = args.backward_tokens or P["T"]
+    T = min(args.backward_tokens, P["T"]) if args.backward_tokens > 0 else P["T"]
     x = {n: inp[n][:, :T].contiguous() for n in ("q", "k", "v", "log_alpha", "beta")}
     x["init_state"] = inp["init_state"]
     head_tokens = P["B"] * T * P["H"]
