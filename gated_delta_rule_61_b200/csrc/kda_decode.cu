@@ -239,6 +239,9 @@ decode_multi_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
   __shared__ float4 s_red[2][kWarps][2][LPR];
   __shared__ __align__(16) float s_fin[2][2][4 * LPR];   // r and p of the CTA's columns
 
+  // programmatic dependent launch: wait for the previous kernel on the stream
+  // (it may update this state) before reading anything
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   float* S = state + (size_t)head * DK * DV;
   float4 s[NI];
 #pragma unroll
@@ -359,6 +362,7 @@ decode_multi_kernel(const TIn* __restrict__ q, const TIn* __restrict__ k,
     const int row = (warp + i * kWarps) * RPI + sub;
     __stcs(reinterpret_cast<float4*>(S + (size_t)row * DV + col), s[i]);
   }
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 template <typename TIn, int DK, int DV, int kSplit>
@@ -366,19 +370,19 @@ static cudaError_t launch_decode_split(const void* q, const void* k, const void*
                                        const float* la, const float* beta, float* state,
                                        void* o, int n_heads, int T, int H, int gate,
                                        unsigned flags, cudaStream_t stream) {
+  // programmatic dependent launch: scheduled while the previous kernel on
+  // the stream finishes (the kernels wait for it before reading anything)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(n_heads * kSplit));
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (T == 1) {
     const bool forms = gate != kGateChannel || flags != 0u;
-    // programmatic dependent launch: scheduled while the previous kernel on
-    // the stream finishes (the kernel waits for it before reading anything)
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(n_heads * kSplit));
-    cfg.blockDim = dim3(256);
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     if (forms)
       return cudaLaunchKernelEx(&cfg, decode_step_kernel<TIn, DK, DV, kSplit, true>,
                                 (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, state,
@@ -387,9 +391,9 @@ static cudaError_t launch_decode_split(const void* q, const void* k, const void*
                               (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, state,
                               (TIn*)o, gate, flags);
   }
-  decode_multi_kernel<TIn, DK, DV, kSplit><<<n_heads * kSplit, 256, 0, stream>>>(
-      (const TIn*)q, (const TIn*)k, (const TIn*)v, la, beta, state, (TIn*)o, T, H, gate, flags);
-  return cudaGetLastError();
+  return cudaLaunchKernelEx(&cfg, decode_multi_kernel<TIn, DK, DV, kSplit>, (const TIn*)q,
+                            (const TIn*)k, (const TIn*)v, la, beta, state, (TIn*)o, T, H, gate,
+                            flags);
 }
 
 // Value slices per head: 2 (dv = 128) or 1 (dv = 64) fill the GPU once there
