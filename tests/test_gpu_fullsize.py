@@ -6,7 +6,8 @@ B=256 H=32 d=128 for 1000 in-place steps: every head's output at every step
 and every head's state after the last step; packed varlen 64 sequences
 log-uniform in [128, 32768] with H=32: every sequence on four heads; long
 prefill T=1,048,576 H=32: the first 16384 tokens of every head, the whole
-sequence against a split prefill, then decode steps. The large inputs are
+sequence against a split prefill, then decode steps; the prefill's other gate
+forms and the fused prologue at its full size, every chain. The large inputs are
 drawn on the GPU by the seeded generator and copied to the host for the
 oracle. Tolerances as in test_gpu_parity (normwise).
 """
@@ -152,3 +153,45 @@ def test_long_context_prefill_then_decode():
         assert_close(s, S_host, TOL_F32, "long-context decode state step %d" % step)
     st, detail = kda.device_status()
     assert st == kda.KDA_OK, (st, detail)
+
+
+@pytest.mark.parametrize("form", ["scalar", "none", "raw"])
+def test_prefill_forms_full_size_every_chain(form):
+    """The other gate forms and the fused prologue at the benchmark's prefill
+    size (B=4 T=8192 H=16, as the benchmark times them): every chain against
+    the oracle. Scalar gate: log sigmoid(N(3, 1)) per (token, head); raw:
+    unnormalised N(0, 1) q and k, beta logits N(0, 1) and gate logits N(3, 1)
+    per key channel, the clamp applied to log sigmoid of the logits."""
+    B, T, H, d = 4, 8192, 16, 128
+    inp = prefill_inputs(B, T, H, d, d, dtype=torch.bfloat16, seed=5, init_std=0.1,
+                         device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(55)
+    gate, raw = {"scalar": ("scalar", False), "none": ("none", False),
+                 "raw": ("channel", True)}[form]
+    q, k, la, beta = inp["q"], inp["k"], inp["log_alpha"], inp["beta"]
+    if form == "scalar":
+        la = torch.nn.functional.logsigmoid(torch.randn(B, T, H, device="cuda", generator=g) + 3.0)
+    elif form == "none":
+        la = None
+    else:
+        q = torch.randn(q.shape, device="cuda", generator=g).to(torch.bfloat16)
+        k = torch.randn(k.shape, device="cuda", generator=g).to(torch.bfloat16)
+        beta = torch.randn(beta.shape, device="cuda", generator=g)
+        la = torch.randn(la.shape, device="cuda", generator=g) + 3.0
+    o, s = kda.prefill(q, k, inp["v"], la, beta, init_state=inp["init_state"], chunk=64,
+                       gate=gate, raw_qk=raw, raw_beta=raw, raw_gate=raw)
+    torch.cuda.synchronize()
+    la_h = None
+    if la is not None:
+        la_h = la.cpu().double()
+        if raw:
+            la_h = torch.from_numpy(oracle.log_sigmoid(la_h))
+        la_h = la_h.clamp(min=CLAMP)
+    o_ref, s_ref = oracle.kda_forward_ex(q.cpu(), k.cpu(), inp["v"].cpu(), la_h, beta.cpu(),
+                                         init_state=inp["init_state"].cpu(), gate=gate,
+                                         raw_qk=raw, raw_beta=raw, raw_gate=False)
+    o_h, s_h = o.cpu(), s.cpu()
+    worst_o = max(normwise(o_h[b, :, h], o_ref[b, :, h]) for b in range(B) for h in range(H))
+    worst_s = max(normwise(s_h[b, h], s_ref[b, h]) for b in range(B) for h in range(H))
+    assert worst_o <= TOL_BF16_O, "%s: o, worst of 64 chains: %.3e" % (form, worst_o)
+    assert worst_s <= TOL_BF16_STATE, "%s: final state, worst of 64 chains: %.3e" % (form, worst_s)
