@@ -7,7 +7,8 @@ and every head's state after the last step; packed varlen 64 sequences
 log-uniform in [128, 32768] with H=32: every sequence on four heads; long
 prefill T=1,048,576 H=32: the first 16384 tokens of every head, the whole
 sequence against a split prefill, then decode steps; the prefill's other gate
-forms and the fused prologue at its full size, every chain. The large inputs are
+forms and the fused prologue at its full size, every chain; 16-token decode
+calls at the decode size; the backward at the prefill size. The large inputs are
 drawn on the GPU by the seeded generator and copied to the host for the
 oracle. Tolerances as in test_gpu_parity (normwise).
 """
@@ -195,3 +196,49 @@ def test_prefill_forms_full_size_every_chain(form):
     worst_s = max(normwise(s_h[b, h], s_ref[b, h]) for b in range(B) for h in range(H))
     assert worst_o <= TOL_BF16_O, "%s: o, worst of 64 chains: %.3e" % (form, worst_o)
     assert worst_s <= TOL_BF16_STATE, "%s: final state, worst of 64 chains: %.3e" % (form, worst_s)
+
+
+def test_multi_token_decode_full_size():
+    """16 tokens per call at the benchmark's decode size (B=256 H=32 d=128,
+    per-channel gate, bf16 inputs): every head's 16 outputs and final state
+    against the oracle's token loop from the same cached state."""
+    B, T, H, d = 256, 16, 32, 128
+    g = torch.Generator(device="cuda").manual_seed(77)
+    x = {n: torch.randn(B, T, H, d, device="cuda", generator=g) for n in ("q", "k", "v")}
+    for n in ("q", "k"):
+        x[n] = x[n] / x[n].norm(dim=-1, keepdim=True)
+    x = {n: t.to(torch.bfloat16) for n, t in x.items()}
+    la = torch.nn.functional.logsigmoid(torch.randn(B, T, H, d, device="cuda", generator=g) + 3.0)
+    b = torch.sigmoid(torch.randn(B, T, H, device="cuda", generator=g))
+    S = decode_state(B, H, d, d, std=0.05, seed=4, device="cuda")
+    S0 = S.cpu()
+    o = kda.decode(x["q"], x["k"], x["v"], la, b, S)
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle.kda_forward(x["q"].cpu(), x["k"].cpu(), x["v"].cpu(), la.cpu(), b.cpu(),
+                                      init_state=S0)
+    assert_close(o.cpu(), o_ref, TOL_BF16_O, "multi-token decode o, all heads")
+    worst_s = max(normwise(S[bb].cpu(), s_ref[bb]) for bb in range(B))
+    assert worst_s <= TOL_F32, "multi-token decode state, worst sequence: %.3e" % worst_s
+
+
+def test_backward_full_size():
+    """The backward at the benchmark's prefill size (B=4 T=8192 H=16, bf16,
+    per-channel gate): every gradient against the oracle's fp64 reverse mode,
+    per (sequence, head) for the state gradient."""
+    B, T, H, d = 4, 8192, 16, 128
+    inp = prefill_inputs(B, T, H, d, d, dtype=torch.bfloat16, seed=6, init_std=0.1,
+                         device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(66)
+    d_o = torch.randn(inp["v"].shape, device="cuda", generator=g).to(torch.bfloat16)
+    d_fin = torch.randn(inp["init_state"].shape, device="cuda", generator=g)
+    out = kda.backward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], d_o,
+                       init_state=inp["init_state"], d_final=d_fin)
+    torch.cuda.synchronize()
+    ref = oracle.kda_backward(inp["q"].cpu(), inp["k"].cpu(), inp["v"].cpu(),
+                              inp["log_alpha"].cpu(), inp["beta"].cpu(), d_o.cpu(),
+                              init_state=inp["init_state"].cpu(), d_final=d_fin.cpu())
+    for n in ("dq", "dk", "dv", "dlog_alpha", "dbeta"):
+        assert_close(out[n].cpu(), ref[n], TOL_F32, "full-size backward %s" % n)
+    worst = max(normwise(out["d_init"][b, h].cpu(), ref["d_init"][b, h])
+                for b in range(B) for h in range(H))
+    assert worst <= TOL_F32, "full-size backward d_init, worst chain: %.3e" % worst
