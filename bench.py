@@ -60,6 +60,16 @@ def peaks():
         return 6650.0, 1590.0, "fallback"
 
 
+def sustained_tflops():
+    """The bf16 GEMM peak measured under the power cap over seconds (the
+    denominator for a kernel timed inside a long loop), or the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops_sustained"])
+    except Exception:
+        return 1400.0
+
+
 def code_hash(path):
     """sha256 (first 16 hex digits) of a CUDA source with comments and
     whitespace removed: a comment edit keeps it, a code change does not."""
@@ -700,7 +710,9 @@ def bench_ours(args):
                          "unit": "GB/s", "frac": achieved_gbs / hbm, "traffic": traffic,
                          "peak_kind": peak_kind, "kernel_ms": kernel_ms,
                          "tensor": {"achieved_tflops": tflops, "peak_tflops": bf16_tf,
-                                    "frac": tflops / bf16_tf}},
+                                    "frac": tflops / bf16_tf,
+                                    "peak_tflops_sustained": sustained_tflops(),
+                                    "frac_sustained": tflops / sustained_tflops()}},
             "decode": dec, "varlen": var, "long": lng, "forms": forms, "backward": bwd, "e2e": e2e,
             "cpu_baseline": cpu,
             "gpu_launches": args.steps, "clocks": clk.summary(),
